@@ -1,0 +1,551 @@
+"""Benchmark of the TPA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Default workload: the 8 x 2048-token prefill of a d_model=1024, h=16, d_h=64,
+R_Q=6, R_K=R_V=2 layer (bf16).  One step = project (+RoPE) -> cache append -> causal
+prefill for the batch, then one decode token per sequence (project the new token,
+append it, decode over 2049 keys), i.e. every step of the hot path once.  The
+value is whole-job algorithmic TFLOP/s.  The same line carries the decode leg on
+the 64 x 32768-token factor cache (GB/s of factor bytes), the roofline of the
+dominant kernel, the fp64 oracle timed on the host cores, an end-to-end number
+through the public API with host buffers, and SM clocks sampled during the timed
+region.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own batch (sequences
+are independent, no data-path collective), so scaling is weak; the time is the max
+over ranks.  `--impl reference` times the fp64 oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from tensor_product_attention_b200 import inputs as I  # noqa: E402
+
+METRIC = "TPA decode factor-cache GB/s (% HBM peak); prefill TFLOP/s (% bf16 peak)"
+DEFAULT = "prefill_b8_s2048_d1024"
+DECODE_LEG = "decode_b64_ctx32k"
+FLUSH_BYTES = 256 << 20          # > 126 MB L2
+
+
+# ------------------------------------------------------------------ accounting
+
+def attn_flops_per_pair(wl) -> int:
+    """Algorithmic flops per (query, key) pair, all heads: the B-space score
+    contraction 2 R_Q R_K d_h, its per-head a_Q a_K weighting 2 h R_Q R_K, and the
+    weighted sum of values 2 h d_h."""
+    return 2 * wl.rank_q * wl.rank_k * wl.head_dim + 2 * wl.n_heads * wl.rank_q * wl.rank_k \
+        + 2 * wl.n_heads * wl.head_dim
+
+
+def proj_flops(wl, tokens: int) -> int:
+    n = (wl.rank_q + wl.rank_k + wl.rank_v) * (wl.n_heads + wl.head_dim)
+    return 2 * tokens * n * wl.d_model
+
+
+def causal_pairs(batch: int, S: int, start: int = 0) -> int:
+    return batch * (S * start + S * (S + 1) // 2)
+
+
+def cache_bytes_per_token(wl) -> int:
+    es = 2 if wl.dtype == "bf16" else 4
+    return (wl.rank_k + wl.rank_v) * (wl.n_heads + wl.head_dim) * es
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+# ------------------------------------------------------------------ helpers
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(ws, value: float) -> float:
+    if ws == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class Events:
+    """CUDA events on the launching stream, one pair per named region per step."""
+
+    def __init__(self):
+        self.pairs = {}
+
+    def start(self, name):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        self.pairs.setdefault(name, []).append([e, None])
+
+    def stop(self, name):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        self.pairs[name][-1][1] = e
+
+    def mean_ms(self, name):
+        v = [a.elapsed_time(b) for a, b in self.pairs.get(name, [])]
+        return sum(v) / len(v) if v else float("nan")
+
+    def total_ms(self, name):
+        return sum(a.elapsed_time(b) for a, b in self.pairs.get(name, []))
+
+
+# ------------------------------------------------------------------ prefill workload
+
+class PrefillStep:
+    """Buffers and the calls of one prefill step (+ one decode token per sequence)."""
+
+    def __init__(self, wl, tpa):
+        self.wl, self.tpa = wl, tpa
+        B, S = wl.batch, wl.seqlen
+        dt = tpa.BF16 if wl.dtype == "bf16" else tpa.F32
+        self.dims = tpa.Dims(wl.d_model, wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v, dt)
+        self.cap = S + 1
+        self.cs = torch.empty((self.cap, wl.head_dim // 2, 2), dtype=torch.float32, device="cuda")
+        tpa.tpa_rope_table(self.dims, wl.rope_base, self.cap, self.cs)
+        self.x_host = torch.cat([I.prefill_x(wl, b) for b in range(B)]).pin_memory()
+        self.xn_host = torch.stack([I.prefill_x(wl, b, S + 1)[S] for b in range(B)]).pin_memory()
+        self.x = self.x_host.cuda()
+        self.xn = self.xn_host.cuda()
+        self.w = I.prefill_w(wl).cuda()
+        self.fac = tpa.alloc_factors(self.dims, B * S)
+        self.fac1 = tpa.alloc_factors(self.dims, B)
+        self.cache = tpa.alloc_cache(self.dims, B, self.cap)
+        tdt = self.dims.torch_dtype
+        self.out = torch.empty((B * S, wl.n_heads, wl.head_dim), dtype=tdt, device="cuda")
+        self.out1 = torch.empty((B, wl.n_heads, wl.head_dim), dtype=tdt, device="cuda")
+        self.lengths = [S + 1] * B
+        self.ws = tpa.alloc_workspace(self.dims, self.lengths)
+        self.out_host = torch.empty(self.out.shape, dtype=tdt).pin_memory()
+        self.out1_host = torch.empty(self.out1.shape, dtype=tdt).pin_memory()
+        self.launches_per_step = 7   # project, append, prefill, project, append, decode, combine
+
+    def flops(self):
+        wl = self.wl
+        B, S = wl.batch, wl.seqlen
+        f = proj_flops(wl, B * (S + 1))
+        f += attn_flops_per_pair(wl) * (causal_pairs(B, S) + B * (S + 1))
+        return f
+
+    def run(self, ev: Events | None = None):
+        t, wl, d = self.tpa, self.wl, self.dims
+        B, S = wl.batch, wl.seqlen
+        zero = [0] * B
+        mark = (lambda n: ev.start(n)) if ev else (lambda n: None)
+        done = (lambda n: ev.stop(n)) if ev else (lambda n: None)
+        mark("project"); t.tpa_project(d, self.x, self.w, B, S, zero, self.cs, self.cap, self.fac); done("project")
+        mark("append"); t.tpa_cache_append(d, self.cache, self.fac, B, S, zero); done("append")
+        mark("prefill"); t.tpa_prefill(d, self.fac, self.cache, B, S, zero, self.out); done("prefill")
+        mark("decode_step")
+        pos = [S] * B
+        t.tpa_project(d, self.xn, self.w, B, 1, pos, self.cs, self.cap, self.fac1)
+        t.tpa_cache_append(d, self.cache, self.fac1, B, 1, pos)
+        t.tpa_decode(d, self.fac1.a_q, self.fac1.b_q, self.cache, self.lengths, self.out1, self.ws)
+        done("decode_step")
+
+    def run_e2e(self):
+        """The same step from pinned host buffers: copy x in, run, copy the outputs out."""
+        self.x.copy_(self.x_host, non_blocking=True)
+        self.xn.copy_(self.xn_host, non_blocking=True)
+        self.run()
+        self.out_host.copy_(self.out, non_blocking=True)
+        self.out1_host.copy_(self.out1, non_blocking=True)
+
+    def io_bytes(self):
+        h2d = self.x_host.numel() * self.x_host.element_size() + self.xn_host.numel() * self.xn_host.element_size()
+        d2h = self.out_host.numel() * self.out_host.element_size() + self.out1_host.numel() * self.out1_host.element_size()
+        return h2d, d2h
+
+
+# ------------------------------------------------------------------ decode workload
+
+class DecodeStep:
+    def __init__(self, wl, tpa):
+        self.wl, self.tpa = wl, tpa
+        self.dims = tpa.Dims(0, wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v,
+                             tpa.BF16 if wl.dtype == "bf16" else tpa.F32)
+        self.lengths = [int(v) for v in I.decode_lengths(wl)]
+        B = wl.batch
+        self.cache = tpa.alloc_cache(self.dims, B, max(self.lengths))
+        qa, qb = [], []
+        for b, L in enumerate(self.lengths):
+            seq = I.decode_sequence(wl, b, L)
+            for n in ("a_k", "a_v", "b_k", "b_v"):
+                getattr(self.cache, n)[b, :L].copy_(seq[n])
+            if wl.rank_q:
+                qa.append(seq["a_q"]); qb.append(seq["b_q"])
+            else:
+                qb.append(seq["q"])
+            del seq
+        self.qa_host = torch.stack(qa).pin_memory() if qa else None
+        self.qb_host = torch.stack(qb).pin_memory()
+        self.q_a = self.qa_host.cuda() if qa else None
+        self.q_b = self.qb_host.cuda()
+        tdt = self.dims.torch_dtype
+        self.out = torch.empty((B, wl.n_heads, wl.head_dim), dtype=tdt, device="cuda")
+        self.out_host = torch.empty(self.out.shape, dtype=tdt).pin_memory()
+        self.ws = tpa.alloc_workspace(self.dims, self.lengths)
+        self.launches_per_step = 2   # decode, combine
+
+    def factor_bytes(self):
+        return sum(self.lengths) * cache_bytes_per_token(self.wl)
+
+    def bytes(self):
+        q = self.q_b.numel() * self.q_b.element_size() + (0 if self.q_a is None else self.q_a.numel() * self.q_a.element_size())
+        return self.factor_bytes() + q + self.out.numel() * self.out.element_size()
+
+    def run(self, ev: Events | None = None):
+        if ev:
+            ev.start("decode")
+        self.tpa.tpa_decode(self.dims, self.q_a, self.q_b, self.cache, self.lengths, self.out, self.ws)
+        if ev:
+            ev.stop("decode")
+
+    def run_e2e(self):
+        if self.q_a is not None:
+            self.q_a.copy_(self.qa_host, non_blocking=True)
+        self.q_b.copy_(self.qb_host, non_blocking=True)
+        self.run()
+        self.out_host.copy_(self.out, non_blocking=True)
+
+    def io_bytes(self):
+        h2d = self.qb_host.numel() * self.qb_host.element_size()
+        if self.qa_host is not None:
+            h2d += self.qa_host.numel() * self.qa_host.element_size()
+        return h2d, self.out_host.numel() * self.out_host.element_size()
+
+
+# ------------------------------------------------------------------ timing
+
+def timed(step, steps, warmup, ws, flush: torch.Tensor | None):
+    """W untimed steps, then exactly K timed steps between barrier+sync; per-step CUDA
+    events on the launching stream (the L2 flush, when used, sits between steps and
+    outside the events).  Returns (per-step ms averaged over K, max over ranks; events)."""
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize()
+    ev = Events()
+    barrier(ws)
+    torch.cuda.synchronize()
+    for _ in range(steps):
+        if flush is not None:
+            flush.zero_()
+        ev.start("step")
+        step.run(ev)
+        ev.stop("step")
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms = ev.total_ms("step") / steps
+    return max_over_ranks(ws, ms), ev
+
+
+def timed_e2e(step, steps, warmup, ws):
+    for _ in range(warmup):
+        step.run_e2e()
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step.run_e2e()
+    b.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    return max_over_ranks(ws, a.elapsed_time(b) / steps)
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_prefill_sample(wl, n_seq: int = 1, seqlen: int | None = None):
+    """Time the oracle's forward (project + RoPE + causal attention, fp64) on n_seq
+    sequences of the workload; returns (seconds, flops of that sample)."""
+    import oracle
+    S = seqlen or wl.seqlen
+    od = oracle.Dims(wl.d_model, wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v)
+    x = np.stack([I.prefill_x(wl, b, S).double().numpy() for b in range(n_seq)])
+    w = I.prefill_w(wl).double().numpy()
+    t0 = time.perf_counter()
+    oracle.tpa_forward(x, w, od, wl.rope_base)
+    dt = time.perf_counter() - t0
+    return dt, proj_flops(wl, n_seq * S) + attn_flops_per_pair(wl) * causal_pairs(n_seq, S)
+
+
+def oracle_decode_sample(wl, n_seq: int = 1, length: int | None = None):
+    """Time the oracle's decode on n_seq sequences; returns (seconds, factor bytes)."""
+    import oracle
+    od = oracle.Dims(0, wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v)
+    lengths = I.decode_lengths(wl)
+    total = 0
+    seqs = []
+    for b in range(n_seq):
+        L = int(length or lengths[b])
+        seqs.append(({k: v.double().numpy() for k, v in I.decode_sequence(wl, b, L).items()}, L))
+        total += L * cache_bytes_per_token(wl)
+    t0 = time.perf_counter()
+    for s, L in seqs:
+        oracle.decode_attention(s, s, od, L)
+    return time.perf_counter() - t0, total
+
+
+def cpu_baseline(wl):
+    if wl.kind == "prefill":
+        dt, fl = oracle_prefill_sample(wl, 1)
+        return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                "sample": f"fp64 oracle forward of 1 of {wl.batch} sequences ({wl.seqlen} tokens): "
+                          f"projection, RoPE, causal attention; {dt:.1f} s"}
+    dt, by = oracle_decode_sample(wl, 2)
+    return {"value": by / dt / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle decode of 2 of {wl.batch} sequences; {dt:.1f} s"}
+
+
+# ------------------------------------------------------------------ main
+
+def run_reference(args, wl, ws, rank):
+    """The fp64 oracle on the host cores, timed per step on a bounded sample."""
+    if rank != 0:
+        return
+    vals = []
+    for _ in range(args.warmup + args.steps):
+        if wl.kind == "prefill":
+            dt, fl = oracle_prefill_sample(wl, 1, seqlen=512)
+            vals.append(fl / dt / 1e12)
+        else:
+            dt, by = oracle_decode_sample(wl, 1, length=8192)
+            vals.append(by / dt / 1e9)
+    v = statistics.mean(vals[args.warmup:])
+    unit = "TFLOP/s" if wl.kind == "prefill" else "GB/s"
+    sample = ("fp64 oracle forward of one 512-token sequence per step" if wl.kind == "prefill"
+              else "fp64 oracle decode of one 8192-token sequence per step")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name},
+        "cpu_baseline": {"value": v, "unit": unit, "cores": cpu_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT, choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode-leg", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = I.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        ws = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, wl, ws, rank)
+        return
+
+    ws, rank, local = dist_setup()
+    from tensor_product_attention_b200 import binding as tpa
+    pk = peaks()
+
+    step = PrefillStep(wl, tpa) if wl.kind == "prefill" else DecodeStep(wl, tpa)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if wl.kind == "prefill" else None
+    with ClockSampler(local) as clk:
+        ms, ev = timed(step, args.steps, args.warmup, ws, flush)
+        e2e_ms = timed_e2e(step, args.steps, args.warmup, ws)
+    clocks = clk.summary()
+    assert tpa.tpa_get_device_error() == 0
+
+    if wl.kind == "prefill":
+        work = step.flops()
+        value = ws * work / (ms * 1e-3) / 1e12
+        e2e_v = ws * work / (e2e_ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        pre_ms = ev.mean_ms("prefill")
+        pre_fl = attn_flops_per_pair(wl) * causal_pairs(wl.batch, wl.seqlen)
+        ach = pre_fl / (pre_ms * 1e-3) / 1e12
+        roof = {"kernel": "tpa_prefill (causal attention from factors)", "bound": "tensor",
+                "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / pk["bf16_tflops"], "traffic": None,
+                "peak_kind": f"bf16 dense, burst, {pk['source']}",
+                "algorithmic_per_launch": f"{pre_fl:.4g} flop = {attn_flops_per_pair(wl)} flop/pair x "
+                                          f"{causal_pairs(wl.batch, wl.seqlen)} causal pairs",
+                "launch_ms": pre_ms}
+        legs = {n: round(ev.mean_ms(n), 4) for n in ("project", "append", "prefill", "decode_step")}
+        config = {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seqlen, "d_model": wl.d_model,
+                  "n_heads": wl.n_heads, "head_dim": wl.head_dim, "rank_q": wl.rank_q,
+                  "rank_k": wl.rank_k, "rank_v": wl.rank_v,
+                  "step": "project+RoPE -> append -> causal prefill, then 1 decode token per sequence",
+                  "l2": "flushed between steps (256 MiB write outside the step events)",
+                  "parallelism": f"dp{ws} (independent sequences per rank)"}
+    else:
+        work = step.bytes()
+        value = ws * work / (ms * 1e-3) / 1e9
+        e2e_v = ws * work / (e2e_ms * 1e-3) / 1e9
+        unit = "GB/s"
+        ach = step.factor_bytes() / (ev.mean_ms("decode") * 1e-3) / 1e9
+        roof = {"kernel": "tpa_decode (split-K decode + combine)", "bound": "hbm", "achieved": ach,
+                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"], "traffic": None,
+                "peak_kind": f"HBM copy, {pk['source']}",
+                "algorithmic_per_launch": f"{step.factor_bytes()} factor bytes",
+                "launch_ms": ev.mean_ms("decode")}
+        legs = {"decode": round(ev.mean_ms("decode"), 4)}
+        config = {"workload": wl.name, "batch": wl.batch, "context": list(wl.context),
+                  "n_heads": wl.n_heads, "head_dim": wl.head_dim, "rank_q": wl.rank_q,
+                  "rank_k": wl.rank_k, "rank_v": wl.rank_v, "l2": "inputs larger than L2",
+                  "parallelism": f"dp{ws} (independent sequences per rank)"}
+    h2d, d2h = step.io_bytes()
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded, workload distributions)",
+        "config": config, "roofline": roof, "legs_ms": legs, "clocks": clocks,
+        "e2e": {"value": e2e_v, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": step.launches_per_step * args.steps,
+    }
+    del step
+    torch.cuda.empty_cache()
+
+    if wl.kind == "prefill" and not args.no_decode_leg:
+        dl = I.WORKLOADS[DECODE_LEG]
+        dstep = DecodeStep(dl, tpa)
+        dms, dev = timed(dstep, args.steps, args.warmup, ws, None)
+        dval = ws * dstep.bytes() / (dms * 1e-3) / 1e9
+        dach = dstep.factor_bytes() / (dev.mean_ms("decode") * 1e-3) / 1e9
+        line["decode_leg"] = {"workload": dl.name, "value": dval, "unit": "GB/s", "ms_per_step": dms,
+                              "frac_of_hbm": dach / pk["hbm_gbs"], "factor_bytes": dstep.factor_bytes(),
+                              "gpu_launches": dstep.launches_per_step * args.steps}
+        line["gpu_launches"] += dstep.launches_per_step * args.steps
+        del dstep
+        torch.cuda.empty_cache()
+
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line))
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

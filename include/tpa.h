@@ -1,0 +1,196 @@
+/*
+ * tpa.h - C ABI of libtpa.so: the data-parallel hot path of Tensor Product Attention
+ * (TPA) on NVIDIA B200 (sm_100a).
+ *
+ * TPA writes each token's query, key and value as a contextual rank-R sum
+ *     Q_t = (1/R_Q) sum_r a_r^Q(x_t) (outer) b_r^Q(x_t),  a_r in R^h, b_r in R^{d_h}
+ * and likewise for K (R_K) and V (R_V)  ["【拜读】Tensor Product Attention Is All You Need
+ * 姚期智团队开源兼容RoPE位置编码" (coreui.cn), 核心机制总结 §3 公式描述].  Only the factors
+ * are cached, B_K already rotated by RoPE at its position [same page, 关键问题及回答 问题2],
+ * and attention softmax(Q K^T / sqrt(d_h)) V ["张量积注意力（TPA）…" (jieyibu.net), Ⅱ.1]
+ * is computed from the cached factors; K and V are never written to device memory.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pointers marked "device" point to device memory of the current CUDA device;
+ *    pointers marked "host" point to host memory read before the call returns.
+ *    The caller owns every buffer; the library allocates nothing and keeps no
+ *    pointer after the call returns.  Its only global state is one 32-bit device
+ *    error word per device (tpa_get_device_error).
+ *  - Every compute call is asynchronous on `stream` (a cudaStream_t; NULL means the
+ *    legacy default stream).  Arguments are validated on the host before any launch;
+ *    a call that returns an error has launched nothing.  TPA_ERR_CUDA means a launch
+ *    failed; the CUDA error is left for cudaGetLastError().
+ *  - Element type: dims->dtype selects fp32 (TPA_F32) or bf16 (TPA_BF16) for every
+ *    factor, cache, query and output buffer of the call; x and w_cat use it too.
+ *    Arithmetic is fp32 (bf16 operands on tensor cores, fp32 accumulation and softmax).
+ *  - Layouts are dense row-major with the shapes given below, T = batch * seqlen tokens
+ *    ordered sequence-major (token t = b * seqlen + i).  The A and B factor layouts
+ *    follow the page's views: A_* is [.., h, R] (head-major) and B_* is [.., R, d_h]
+ *    [review, 代码 前向传播].  Device pointers must be 16-byte aligned.
+ *  - Factors are stored raw, without the 1/R; attention applies 1/R_Q, 1/R_K, 1/R_V
+ *    and 1/sqrt(d_h).  B_Q and B_K leave tpa_project already rotated.
+ *  - RoPE: interleaved pairs (2k, 2k+1) of the head dimension turn by p * theta_k,
+ *    theta_k = base^(-2k/d_h), p the 0-based absolute position (the LLaMA convention
+ *    behind the page's freqs_cis / apply_rotary_emb, whose body the pages do not print).
+ *  - Kernels never trap.  Where a kernel waits on a barrier it gives up after a bounded
+ *    number of tries, records TPA_DEVERR_TIMEOUT in the device error word and returns.
+ */
+#ifndef TPA_H
+#define TPA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TPA_ABI_VERSION 1
+#define TPA_MAX_BATCH 1024          /* sequences per call */
+
+typedef struct CUstream_st* tpa_stream_t;   /* same type as cudaStream_t */
+
+typedef enum tpa_status {
+    TPA_OK = 0,
+    TPA_ERR_INVALID = 1,        /* null pointer, bad size, misaligned pointer, bad position */
+    TPA_ERR_UNSUPPORTED = 2,    /* valid TPA shape that no kernel here implements */
+    TPA_ERR_CAPACITY = 3,       /* write past the cache capacity or the RoPE table */
+    TPA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+    TPA_ERR_WORKSPACE = 5,      /* workspace too small */
+    TPA_ERR_DEVICE = 6          /* tpa_get_device_error found a recorded device error */
+} tpa_status;
+
+typedef enum tpa_dtype { TPA_F32 = 0, TPA_BF16 = 1 } tpa_dtype;
+
+/* device error word values (tpa_get_device_error) */
+#define TPA_DEVERR_NONE 0
+#define TPA_DEVERR_TIMEOUT 1        /* a bounded wait gave up */
+#define TPA_DEVERR_BOUNDS 2         /* an index check failed (debug builds) */
+
+/* Shape of one TPA layer: the page's ModelArgs (dim, n_heads, head_dim, q_rank, rank)
+ * [review, 代码 类定义与初始化], with rank split into rank_k and rank_v.
+ * rank_q = 0 selects TPA-KVonly: the query is a plain per-head vector [h][d_h]
+ * (decode only in this version). */
+typedef struct tpa_dims {
+    int32_t d_model;
+    int32_t n_heads;     /* h */
+    int32_t head_dim;    /* d_h, even */
+    int32_t rank_q;      /* R_Q (0: KV-only) */
+    int32_t rank_k;      /* R_K */
+    int32_t rank_v;      /* R_V */
+    int32_t dtype;       /* tpa_dtype */
+} tpa_dims;
+
+/* The six factor tensors of T tokens (device):
+ *   a_q [T][h][R_Q]   a_k [T][h][R_K]   a_v [T][h][R_V]
+ *   b_q [T][R_Q][d_h] b_k [T][R_K][d_h] b_v [T][R_V][d_h]   (b_q, b_k rotated) */
+typedef struct tpa_factors {
+    void* a_q; void* b_q;
+    void* a_k; void* b_k;
+    void* a_v; void* b_v;
+} tpa_factors;
+
+/* The factor cache of `batch` sequences with room for `capacity` tokens each (device),
+ * the page's cache_kA / cache_vA / cache_kB / cache_vB [review, 类定义与初始化]:
+ *   a_k, a_v [batch][capacity][h][R]    b_k, b_v [batch][capacity][R][d_h]
+ * lengths [batch] int32 (device) is written by tpa_cache_append. */
+typedef struct tpa_cache {
+    void* a_k; void* a_v;
+    void* b_k; void* b_v;
+    int32_t* lengths;
+    int32_t batch;
+    int32_t capacity;
+} tpa_cache;
+
+/* ABI version (TPA_ABI_VERSION) and a short description of the library build. */
+int32_t tpa_abi_version(void);
+const char* tpa_build_info(void);
+const char* tpa_status_string(tpa_status status);
+
+/* Bytes the factor cache holds per token: (R_K + R_V) * (h + d_h) * sizeof(element),
+ * from the page's cache shapes [review, 类定义与初始化].  0 for invalid dims. */
+size_t tpa_cache_bytes_per_token(const tpa_dims* dims);
+
+/* RoPE table: cs[p][k][0] = cos(p * theta_k), cs[p][k][1] = sin(p * theta_k) for
+ * p < max_pos, k < d_h/2, angles formed and evaluated in fp64, stored as fp32.
+ * cs: device float [max_pos][d_h/2][2].  This is the caller-supplied freqs_cis of
+ * the page's forward(x, start_pos, freqs_cis, mask) [review, 代码 前向传播]. */
+tpa_status tpa_rope_table(const tpa_dims* dims, double base, int32_t max_pos,
+                          float* cs, tpa_stream_t stream);
+
+/* Factor projection: Y = x W_cat^T, cut into the six factors, with RoPE applied to
+ * the B_Q and B_K columns of token t = b*seqlen+i at position start_pos[b] + i.
+ * The six bias-free projections W_A_q/k/v, W_B_q/k/v of [review, 类定义与初始化 /
+ * 前向传播], fused into one GEMM; RoPE on B before caching per [review, 问题2].
+ *   x      device [T][d_model]
+ *   w_cat  device [N][d_model], N = h(R_Q+R_K+R_V) + d_h(R_Q+R_K+R_V): the six
+ *          nn.Linear weights stacked in the order W_A_q, W_A_k, W_A_v, W_B_q, W_B_k, W_B_v
+ *   start_pos host [batch]; every start_pos[b] + seqlen <= max_pos (else TPA_ERR_CAPACITY)
+ *   rope_cs device table from tpa_rope_table with the same head_dim and >= max_pos rows
+ *   out    device factor buffers for T tokens (all six set, none aliasing x or w_cat)
+ * rank_q = 0 is TPA_ERR_UNSUPPORTED. */
+tpa_status tpa_project(const tpa_dims* dims, const void* x, const void* w_cat,
+                       int32_t batch, int32_t seqlen, const int32_t* start_pos,
+                       const float* rope_cs, int32_t max_pos,
+                       const tpa_factors* out, tpa_stream_t stream);
+
+/* Cache append: for every sequence b and i < n_tokens, copy token b*n_tokens+i of
+ * kv->a_k, kv->a_v, kv->b_k, kv->b_v into cache position start_pos[b] + i, bit for
+ * bit, and set cache->lengths[b] = start_pos[b] + n_tokens.  The page's
+ * cache[:bsz, start_pos:start_pos+seqlen] = factors [review, 代码 前向传播].
+ *   kv         device factors for batch*n_tokens tokens (a_q, b_q ignored)
+ *   start_pos  host [batch]; start_pos[b] + n_tokens <= capacity (else TPA_ERR_CAPACITY)
+ * batch <= cache->batch; sequences >= batch are left alone. */
+tpa_status tpa_cache_append(const tpa_dims* dims, const tpa_cache* cache,
+                            const tpa_factors* kv, int32_t batch, int32_t n_tokens,
+                            const int32_t* start_pos, tpa_stream_t stream);
+
+/* Causal prefill from factors: query i of sequence b (position p = start_pos[b] + i)
+ * attends to cached keys 0..p of sequence b:
+ *   out[b*seqlen+i][h][:] = sum_j softmax_j(q_h . k_{j,h} / sqrt(d_h)) v_{j,h}
+ * with q, k, v the (1/R) rank sums of the factors [review, §3 公式描述 and 前向传播;
+ * jieyibu.net page, Ⅱ.1], evaluated from the factors without writing K or V out.
+ *   q      device a_q, b_q (rotated) for batch*seqlen tokens (other members ignored)
+ *   cache  must already hold positions 0 .. start_pos[b]+seqlen-1 of each sequence
+ *   start_pos host [batch]
+ *   out    device [batch*seqlen][h][d_h] */
+tpa_status tpa_prefill(const tpa_dims* dims, const tpa_factors* q, const tpa_cache* cache,
+                       int32_t batch, int32_t seqlen, const int32_t* start_pos,
+                       void* out, tpa_stream_t stream);
+
+/* Decode: one query per sequence at position lengths[b]-1 attends to cached keys
+ * 0..lengths[b]-1 (the new token is appended first: the page writes the cache before
+ * reading it [review, 代码 前向传播]).  Keys are read only as factors, B_K used as cached
+ * (pre-rotated, so decode rotates nothing [review, 问题2]).  The context is split
+ * across CTAs and the partial softmax states are merged in a fixed order, so results
+ * are run-to-run identical.
+ *   q_a      device [batch][h][R_Q] (NULL when rank_q == 0)
+ *   q_b      device [batch][R_Q][d_h] rotated at lengths[b]-1, or the rotated per-head
+ *            query [batch][h][d_h] when rank_q == 0 (TPA-KVonly)
+ *   lengths  host [batch], 1 <= lengths[b] <= capacity
+ *   out      device [batch][h][d_h]
+ *   workspace device scratch of at least tpa_decode_workspace_bytes() bytes, 256-byte
+ *            aligned; contents on entry do not matter and are undefined on return. */
+tpa_status tpa_decode(const tpa_dims* dims, const void* q_a, const void* q_b,
+                      const tpa_cache* cache, const int32_t* lengths, int32_t batch,
+                      void* out, void* workspace, size_t workspace_bytes,
+                      tpa_stream_t stream);
+
+/* Workspace bytes tpa_decode needs for these lengths (0 for invalid arguments). */
+size_t tpa_decode_workspace_bytes(const tpa_dims* dims, const int32_t* lengths, int32_t batch);
+
+/* Synchronise `stream`, then read and clear the device error word of the current
+ * device.  *code receives the TPA_DEVERR_* value (NULL allowed).  Returns TPA_OK if
+ * it was clear, TPA_ERR_DEVICE if a kernel recorded an error, TPA_ERR_CUDA if the
+ * synchronisation itself failed. */
+tpa_status tpa_get_device_error(tpa_stream_t stream, int32_t* code);
+
+/* Test hook: the number of polls a bounded wait makes before it gives up
+ * (0 restores the default).  Host-side setting, read at each launch. */
+void tpa_set_wait_limit(uint32_t polls);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TPA_H */

@@ -290,3 +290,23 @@ def decode_attention(q_factors: dict, kv: dict, dims: Dims, length: int,
         v = materialize(np.asarray(kv["a_v"][j0:j1]), np.asarray(kv["b_v"][j0:j1]), dims.rank_v)
         out += np.einsum("hl,lhd->hd", p[:, j0:j1], v)
     return out
+
+
+def tpa_forward_rows(x: np.ndarray, w_cat: np.ndarray, dims: Dims, rope_base: float,
+                     rows) -> np.ndarray:
+    """``tpa_forward`` for one sequence that starts at position 0, evaluated only for
+    the query rows ``rows`` (the keys and values still cover the whole sequence), so
+    that long sequences can be checked on a sample of their outputs.
+
+    x: [S, d_model].  Returns out [len(rows), h, d].  Same steps, same order as
+    ``tpa_forward``: project, materialise, rotate the materialised q and k, attend.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    rows = np.asarray(rows).reshape(-1)
+    f = project(x, w_cat, dims)
+    q = materialize(f["a_q"][rows], f["b_q"][rows], dims.rank_q)
+    k = materialize(f["a_k"], f["b_k"], dims.rank_k)
+    v = materialize(f["a_v"], f["b_v"], dims.rank_v)
+    q = rope_rotate(q, rows, rope_base)
+    k = rope_rotate(k, np.arange(x.shape[0]), rope_base)
+    return causal_attention(q, k, v, rows)

@@ -1,0 +1,246 @@
+// The C ABI of libtpa.so (declared in include/tpa.h): host-side validation, the
+// per-device error word, and dispatch to the kernels.  No call allocates memory.
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "tpa_internal.h"
+
+namespace tpa {
+// One error word per device; kernels record the first failure here (never trap).
+__device__ int g_device_error;
+}  // namespace tpa
+
+using namespace tpa;
+
+namespace {
+
+std::atomic<uint32_t> g_wait_limit{0};
+constexpr uint32_t kDefaultWaitLimit = 1u << 26;   // polls, roughly seconds of waiting
+constexpr int kMaxDevices = 64;
+std::mutex g_err_mu;
+int* g_err_ptr[kMaxDevices] = {};
+
+uint32_t wait_limit() {
+    uint32_t v = g_wait_limit.load(std::memory_order_relaxed);
+    return v ? v : kDefaultWaitLimit;
+}
+
+// Device address of the error word on the current device (looked up once per device).
+int* device_error_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_err_mu);
+    if (!g_err_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<int*>(p);
+    }
+    return g_err_ptr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks common to all calls.  need_q: the call reads factorised queries.
+tpa_status check_dims(const tpa_dims* d, bool need_q) {
+    if (!d) return TPA_ERR_INVALID;
+    if (d->dtype != TPA_F32 && d->dtype != TPA_BF16) return TPA_ERR_INVALID;
+    if (d->n_heads < 1 || d->head_dim < 2 || (d->head_dim & 1)) return TPA_ERR_INVALID;
+    if (d->rank_k < 1 || d->rank_v < 1 || d->rank_q < 0) return TPA_ERR_INVALID;
+    if (need_q && d->rank_q < 1) return TPA_ERR_UNSUPPORTED;
+    if (d->n_heads > 4096 || d->head_dim > 4096 || d->rank_q > 256 || d->rank_k > 256 ||
+        d->rank_v > 256)
+        return TPA_ERR_UNSUPPORTED;
+    return TPA_OK;
+}
+
+tpa_status check_cache(const tpa_cache* c, int batch) {
+    if (!c || !c->a_k || !c->a_v || !c->b_k || !c->b_v || !c->lengths) return TPA_ERR_INVALID;
+    if (!aligned16(c->a_k) || !aligned16(c->a_v) || !aligned16(c->b_k) || !aligned16(c->b_v))
+        return TPA_ERR_INVALID;
+    if (c->capacity < 1 || c->batch < 1 || batch < 1 || batch > c->batch ||
+        batch > TPA_MAX_BATCH)
+        return TPA_ERR_INVALID;
+    return TPA_OK;
+}
+
+tpa_status launched(cudaError_t e) { return e == cudaSuccess ? TPA_OK : TPA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t tpa_abi_version(void) { return TPA_ABI_VERSION; }
+
+const char* tpa_build_info(void) {
+    return "libtpa: TPA hot path for sm_100a (tcgen05/TMA kernels for bf16, CUDA-core "
+           "kernels for fp32)";
+}
+
+const char* tpa_status_string(tpa_status s) {
+    switch (s) {
+        case TPA_OK: return "ok";
+        case TPA_ERR_INVALID: return "invalid argument";
+        case TPA_ERR_UNSUPPORTED: return "unsupported shape";
+        case TPA_ERR_CAPACITY: return "position beyond cache capacity or RoPE table";
+        case TPA_ERR_CUDA: return "CUDA error";
+        case TPA_ERR_WORKSPACE: return "workspace too small";
+        case TPA_ERR_DEVICE: return "device-side error recorded";
+    }
+    return "unknown status";
+}
+
+size_t tpa_cache_bytes_per_token(const tpa_dims* d) {
+    if (check_dims(d, false) != TPA_OK) return 0;
+    size_t es = d->dtype == TPA_BF16 ? 2 : 4;
+    return (size_t)(d->rank_k + d->rank_v) * (size_t)(d->n_heads + d->head_dim) * es;
+}
+
+void tpa_set_wait_limit(uint32_t polls) { g_wait_limit.store(polls); }
+
+tpa_status tpa_rope_table(const tpa_dims* d, double base, int32_t max_pos, float* cs,
+                          tpa_stream_t stream) {
+    tpa_status st = check_dims(d, false);
+    if (st != TPA_OK) return st;
+    if (!cs || !aligned16(cs) || max_pos < 1 || !(base > 1.0)) return TPA_ERR_INVALID;
+    if ((long long)max_pos * d->head_dim > (1LL << 34)) return TPA_ERR_UNSUPPORTED;
+    return launched(launch_rope_table(cs, max_pos, d->head_dim, base, (cudaStream_t)stream));
+}
+
+tpa_status tpa_project(const tpa_dims* d, const void* x, const void* w_cat, int32_t batch,
+                       int32_t seqlen, const int32_t* start_pos, const float* rope_cs,
+                       int32_t max_pos, const tpa_factors* out, tpa_stream_t stream) {
+    tpa_status st = check_dims(d, true);
+    if (st != TPA_OK) return st;
+    if (d->d_model < 1) return TPA_ERR_INVALID;
+    if (!x || !w_cat || !start_pos || !rope_cs || !out) return TPA_ERR_INVALID;
+    if (!out->a_q || !out->b_q || !out->a_k || !out->b_k || !out->a_v || !out->b_v)
+        return TPA_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(w_cat) || !aligned16(rope_cs)) return TPA_ERR_INVALID;
+    if (batch < 1 || batch > TPA_MAX_BATCH || seqlen < 1 || max_pos < 1)
+        return TPA_ERR_INVALID;
+    if ((long long)batch * seqlen > (1LL << 30)) return TPA_ERR_UNSUPPORTED;
+    // B_Q / B_K segments must start on an even column so RoPE pairs stay together
+    if ((d->n_heads * (d->rank_q + d->rank_k + d->rank_v)) & 1) return TPA_ERR_UNSUPPORTED;
+    SeqParams sp;
+    for (int b = 0; b < batch; ++b) {
+        if (start_pos[b] < 0) return TPA_ERR_INVALID;
+        if ((long long)start_pos[b] + seqlen > max_pos) return TPA_ERR_CAPACITY;
+        sp.v[b] = start_pos[b];
+    }
+    Shape s = shape_of(*d);
+    ProjLayout L = proj_layout(s, *out);
+    cudaStream_t cs = (cudaStream_t)stream;
+    if (s.bf16 && project_tc_supported(s, batch * seqlen))
+        return launched(launch_project_tc(s, x, w_cat, batch, seqlen, sp, rope_cs, L,
+                                          device_error_ptr(), wait_limit(), cs));
+    return launched(launch_project_simt(s, x, w_cat, batch, seqlen, sp, rope_cs, L, cs));
+}
+
+tpa_status tpa_cache_append(const tpa_dims* d, const tpa_cache* c, const tpa_factors* kv,
+                            int32_t batch, int32_t n_tokens, const int32_t* start_pos,
+                            tpa_stream_t stream) {
+    tpa_status st = check_dims(d, false);
+    if (st != TPA_OK) return st;
+    if ((st = check_cache(c, batch)) != TPA_OK) return st;
+    if (!kv || !kv->a_k || !kv->a_v || !kv->b_k || !kv->b_v || !start_pos)
+        return TPA_ERR_INVALID;
+    if (!aligned16(kv->a_k) || !aligned16(kv->a_v) || !aligned16(kv->b_k) ||
+        !aligned16(kv->b_v))
+        return TPA_ERR_INVALID;
+    if (n_tokens < 1) return TPA_ERR_INVALID;
+    SeqParams sp;
+    for (int b = 0; b < batch; ++b) {
+        if (start_pos[b] < 0) return TPA_ERR_INVALID;
+        if ((long long)start_pos[b] + n_tokens > c->capacity) return TPA_ERR_CAPACITY;
+        sp.v[b] = start_pos[b];
+    }
+    return launched(launch_cache_append(shape_of(*d), *c, *kv, batch, n_tokens, sp,
+                                        (cudaStream_t)stream));
+}
+
+tpa_status tpa_prefill(const tpa_dims* d, const tpa_factors* q, const tpa_cache* c,
+                       int32_t batch, int32_t seqlen, const int32_t* start_pos, void* out,
+                       tpa_stream_t stream) {
+    tpa_status st = check_dims(d, true);
+    if (st != TPA_OK) return st;
+    if ((st = check_cache(c, batch)) != TPA_OK) return st;
+    if (!q || !q->a_q || !q->b_q || !start_pos || !out) return TPA_ERR_INVALID;
+    if (!aligned16(q->a_q) || !aligned16(q->b_q) || !aligned16(out)) return TPA_ERR_INVALID;
+    if (seqlen < 1) return TPA_ERR_INVALID;
+    if (d->head_dim > 256) return TPA_ERR_UNSUPPORTED;
+    SeqParams sp;
+    for (int b = 0; b < batch; ++b) {
+        if (start_pos[b] < 0) return TPA_ERR_INVALID;
+        if ((long long)start_pos[b] + seqlen > c->capacity) return TPA_ERR_CAPACITY;
+        sp.v[b] = start_pos[b];
+    }
+    Shape s = shape_of(*d);
+    cudaStream_t cs = (cudaStream_t)stream;
+    if (s.bf16 && prefill_tc_supported(s))
+        return launched(launch_prefill_tc(s, *q, *c, batch, seqlen, sp, out,
+                                          device_error_ptr(), wait_limit(), cs));
+    return launched(launch_prefill_simt(s, *q, *c, batch, seqlen, sp, out, cs));
+}
+
+size_t tpa_decode_workspace_bytes(const tpa_dims* d, const int32_t* lengths, int32_t batch) {
+    if (check_dims(d, false) != TPA_OK || !lengths || batch < 1 || batch > TPA_MAX_BATCH)
+        return 0;
+    for (int b = 0; b < batch; ++b)
+        if (lengths[b] < 1) return 0;
+    Shape s = shape_of(*d);
+    return decode_workspace_bytes(s, decode_schedule(s, lengths, batch), batch);
+}
+
+tpa_status tpa_decode(const tpa_dims* d, const void* q_a, const void* q_b,
+                      const tpa_cache* c, const int32_t* lengths, int32_t batch, void* out,
+                      void* workspace, size_t workspace_bytes, tpa_stream_t stream) {
+    tpa_status st = check_dims(d, false);
+    if (st != TPA_OK) return st;
+    if ((st = check_cache(c, batch)) != TPA_OK) return st;
+    if (!q_b || !lengths || !out || !workspace) return TPA_ERR_INVALID;
+    if (d->rank_q > 0 && (!q_a || !aligned16(q_a))) return TPA_ERR_INVALID;
+    if (!aligned16(q_b) || !aligned16(out) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return TPA_ERR_INVALID;
+    SeqParams sp;
+    for (int b = 0; b < batch; ++b) {
+        if (lengths[b] < 1) return TPA_ERR_INVALID;
+        if (lengths[b] > c->capacity) return TPA_ERR_CAPACITY;
+        sp.v[b] = lengths[b];
+    }
+    Shape s = shape_of(*d);
+    DecodeSchedule sch = decode_schedule(s, lengths, batch);
+    if (decode_workspace_bytes(s, sch, batch) > workspace_bytes) return TPA_ERR_WORKSPACE;
+    cudaStream_t cs = (cudaStream_t)stream;
+    float* ws = static_cast<float*>(workspace);
+    cudaError_t e;
+    if (s.bf16 && decode_tc_supported(s)) {
+        e = launch_decode_tc(s, q_a, q_b, *c, sp, batch, sch, ws, device_error_ptr(),
+                             wait_limit(), cs);
+    } else {
+        if ((long long)s.H * s.Dh > 8192) return TPA_ERR_UNSUPPORTED;
+        e = launch_decode_simt(s, q_a, q_b, *c, sp, batch, sch, ws, cs);
+    }
+    if (e != cudaSuccess) return TPA_ERR_CUDA;
+    return launched(launch_decode_combine(s, sp, batch, sch, ws, out, cs));
+}
+
+tpa_status tpa_get_device_error(tpa_stream_t stream, int32_t* code) {
+    if (code) *code = 0;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return TPA_ERR_CUDA;
+    int* p = device_error_ptr();
+    if (!p) return TPA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return TPA_ERR_CUDA;
+    if (v != 0) {
+        int zero = 0;
+        if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+            return TPA_ERR_CUDA;
+    }
+    if (code) *code = v;
+    return v ? TPA_ERR_DEVICE : TPA_OK;
+}
+
+}  // extern "C"

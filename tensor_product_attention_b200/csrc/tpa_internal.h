@@ -1,0 +1,94 @@
+// Internal interface between the C ABI (tpa_api.cu) and the kernels.  Not installed.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/tpa.h"
+
+namespace tpa {
+
+// Per-sequence host values (start positions or lengths), passed by value as a kernel
+// parameter so that no device copy (and no allocation) is needed.
+struct SeqParams {
+    int32_t v[TPA_MAX_BATCH];
+};
+
+struct Shape {
+    int D, H, Dh, Rq, Rk, Rv;
+    bool bf16;
+};
+
+inline Shape shape_of(const tpa_dims& d) {
+    return Shape{d.d_model, d.n_heads, d.head_dim, d.rank_q, d.rank_k, d.rank_v,
+                 d.dtype == TPA_BF16};
+}
+
+// Column layout of the stacked projection output: [a_q | a_k | a_v | b_q | b_k | b_v].
+struct ProjLayout {
+    int off[7];    // segment starts, off[6] = N
+    void* dst[6];  // a_q, a_k, a_v, b_q, b_k, b_v
+};
+
+inline ProjLayout proj_layout(const Shape& s, const tpa_factors& f) {
+    ProjLayout L;
+    int w[6] = {s.H * s.Rq, s.H * s.Rk, s.H * s.Rv, s.Rq * s.Dh, s.Rk * s.Dh, s.Rv * s.Dh};
+    L.off[0] = 0;
+    for (int i = 0; i < 6; ++i) L.off[i + 1] = L.off[i] + w[i];
+    L.dst[0] = f.a_q; L.dst[1] = f.a_k; L.dst[2] = f.a_v;
+    L.dst[3] = f.b_q; L.dst[4] = f.b_k; L.dst[5] = f.b_v;
+    return L;
+}
+
+// Decode split schedule: sequence b is cut into ceil(len_b / split_len) pieces.
+struct DecodeSchedule {
+    int split_len;      // keys per split (multiple of the kernel's key tile)
+    int max_splits;     // grid.x
+};
+
+DecodeSchedule decode_schedule(const Shape& s, const int32_t* lengths, int batch);
+size_t decode_workspace_bytes(const Shape& s, const DecodeSchedule& sch, int batch);
+
+// ---- launchers (each returns the launch's cudaError_t) ----
+cudaError_t launch_rope_table(float* cs, int max_pos, int head_dim, double base,
+                              cudaStream_t st);
+
+cudaError_t launch_project_simt(const Shape& s, const void* x, const void* w, int batch,
+                                int seqlen, const SeqParams& start, const float* cs,
+                                const ProjLayout& L, cudaStream_t st);
+
+cudaError_t launch_project_tc(const Shape& s, const void* x, const void* w, int batch,
+                              int seqlen, const SeqParams& start, const float* cs,
+                              const ProjLayout& L, int* err, uint32_t wait_limit,
+                              cudaStream_t st);
+bool project_tc_supported(const Shape& s, int T);
+
+cudaError_t launch_cache_append(const Shape& s, const tpa_cache& c, const tpa_factors& kv,
+                                int batch, int n_tokens, const SeqParams& start,
+                                cudaStream_t st);
+
+cudaError_t launch_prefill_simt(const Shape& s, const tpa_factors& q, const tpa_cache& c,
+                                int batch, int seqlen, const SeqParams& start, void* out,
+                                cudaStream_t st);
+
+cudaError_t launch_prefill_tc(const Shape& s, const tpa_factors& q, const tpa_cache& c,
+                              int batch, int seqlen, const SeqParams& start, void* out,
+                              int* err, uint32_t wait_limit, cudaStream_t st);
+bool prefill_tc_supported(const Shape& s);
+
+cudaError_t launch_decode_simt(const Shape& s, const void* q_a, const void* q_b,
+                               const tpa_cache& c, const SeqParams& len, int batch,
+                               const DecodeSchedule& sch, float* ws, cudaStream_t st);
+
+cudaError_t launch_decode_tc(const Shape& s, const void* q_a, const void* q_b,
+                             const tpa_cache& c, const SeqParams& len, int batch,
+                             const DecodeSchedule& sch, float* ws, int* err,
+                             uint32_t wait_limit, cudaStream_t st);
+bool decode_tc_supported(const Shape& s);
+
+cudaError_t launch_decode_combine(const Shape& s, const SeqParams& len, int batch,
+                                  const DecodeSchedule& sch, const float* ws, void* out,
+                                  cudaStream_t st);
+
+}  // namespace tpa

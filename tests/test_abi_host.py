@@ -1,0 +1,98 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol tpa.h
+declares, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tpa.h")
+
+
+@pytest.fixture(scope="module")
+def bnd():
+    from tensor_product_attention_b200 import build
+    build.build()
+    from tensor_product_attention_b200 import binding
+    return binding
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tpa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_what_binding_wraps(bnd):
+    assert declared_functions() == sorted(bnd.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(bnd):
+    lib = ctypes.CDLL(bnd.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_abi_version_and_status_strings(bnd):
+    assert bnd.tpa_abi_version() == 1
+    assert "sm_100a" in bnd.tpa_build_info()
+    for code in range(7):
+        assert bnd._lib.tpa_status_string(code)
+
+
+def test_cache_bytes_per_token_matches_golden(bnd):
+    gold = json.load(open(os.path.join(ROOT, "tests", "golden", "cache_bytes_per_token.json")))
+    for row in gold["rows"]:
+        dt = bnd.F32 if row["elem_bytes"] == 4 else bnd.BF16
+        dims = bnd.Dims(64, row["n_heads"], row["head_dim"], 2, row["rank_k"], row["rank_v"], dt)
+        assert bnd.tpa_cache_bytes_per_token(dims) == row["bytes_per_token"]
+    assert bnd.tpa_cache_bytes_per_token(bnd.Dims(64, 4, 15, 2, 1, 1)) == 0   # odd head_dim
+
+
+def _call(bnd, name, *args):
+    return getattr(bnd._lib, name)(*args)
+
+
+def test_host_validation_rejects_bad_arguments(bnd):
+    d = bnd.Dims(64, 4, 16, 2, 1, 1, bnd.F32).c()
+    by = ctypes.byref
+    fake = 0x10000                       # aligned, never dereferenced: validation fails first
+    f = bnd.tpa_factors(fake, fake, fake, fake, fake, fake)
+    c = bnd.tpa_cache(fake, fake, fake, fake, fake, 2, 8)
+    sp = bnd._ints([0, 0])
+    # null pointers
+    assert _call(bnd, "tpa_project", by(d), None, fake, 2, 4, sp, fake, 8, by(f), None) == 1
+    assert _call(bnd, "tpa_prefill", by(d), None, by(c), 2, 4, sp, fake, None) == 1
+    assert _call(bnd, "tpa_decode", by(d), fake, None, by(c), bnd._ints([1, 1]), 2, fake, fake, 1 << 20, None) == 1
+    # misaligned pointer
+    assert _call(bnd, "tpa_project", by(d), fake + 2, fake, 2, 4, sp, fake, 8, by(f), None) == 1
+    # positions past the RoPE table / the cache
+    assert _call(bnd, "tpa_project", by(d), fake, fake, 2, 4, bnd._ints([0, 5]), fake, 8, by(f), None) == 3
+    assert _call(bnd, "tpa_cache_append", by(d), by(c), by(f), 2, 4, bnd._ints([0, 5]), None) == 3
+    assert _call(bnd, "tpa_prefill", by(d), by(f), by(c), 2, 4, bnd._ints([5, 0]), fake, None) == 3
+    assert _call(bnd, "tpa_decode", by(d), fake, fake, by(c), bnd._ints([9, 1]), 2, fake, fake, 1 << 20, None) == 3
+    # batch larger than the cache, zero-length decode, negative start
+    assert _call(bnd, "tpa_cache_append", by(d), by(c), by(f), 3, 1, bnd._ints([0, 0, 0]), None) == 1
+    assert _call(bnd, "tpa_decode", by(d), fake, fake, by(c), bnd._ints([0, 1]), 2, fake, fake, 1 << 20, None) == 1
+    assert _call(bnd, "tpa_cache_append", by(d), by(c), by(f), 2, 1, bnd._ints([-1, 0]), None) == 1
+    # workspace too small
+    need = bnd.tpa_decode_workspace_bytes(bnd.Dims(64, 4, 16, 2, 1, 1, bnd.F32), [3, 5])
+    assert need > 0
+    assert _call(bnd, "tpa_decode", by(d), fake, fake, by(c), bnd._ints([3, 5]), 2, fake, fake, need - 4, None) == 5
+    # bad dims: odd head_dim, zero rank, factorised-query call with rank_q = 0
+    bad = bnd.Dims(64, 4, 15, 2, 1, 1, bnd.F32).c()
+    assert _call(bnd, "tpa_cache_append", by(bad), by(c), by(f), 2, 1, sp, None) == 1
+    kvonly = bnd.Dims(64, 4, 16, 0, 1, 1, bnd.F32).c()
+    assert _call(bnd, "tpa_prefill", by(kvonly), by(f), by(c), 2, 1, sp, fake, None) == 2
+    assert _call(bnd, "tpa_rope_table", by(d), 0.5, 8, fake, None) == 1
+
+
+def test_workspace_size_formula(bnd):
+    dims = bnd.Dims(0, 16, 128, 6, 2, 2)
+    lengths = [32768] * 64
+    n = bnd.tpa_decode_workspace_bytes(dims, lengths)
+    # one (m, l) pair and one d_h-vector of fp32 per (sequence, split, head)
+    per_split = 16 * (128 + 2) * 4
+    assert n % (64 * per_split) == 0 and n > 0

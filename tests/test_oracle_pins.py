@@ -391,3 +391,13 @@ def test_planted_mistakes_are_caught(monkeypatch):
         return out
     assert _pins_fail(monkeypatch, "split_factors", transposed_view,
                       [test_projection_matches_six_separate_linears]) == 1
+
+
+def test_forward_rows_equals_forward():
+    g = gen(17)
+    dims = Dims(d_model=16, n_heads=2, head_dim=8, rank_q=2, rank_k=2, rank_v=1)
+    x = g.standard_normal((1, 21, 16))
+    w = g.standard_normal((sum(oracle.factor_widths(dims).values()), 16)) / 4
+    full, _ = oracle.tpa_forward(x, w, dims, 1e4)
+    rows = [0, 5, 20]
+    assert rel(oracle.tpa_forward_rows(x[0], w, dims, 1e4, rows), full[0, rows]) < 1e-13
