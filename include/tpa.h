@@ -180,6 +180,23 @@ tpa_status tpa_decode(const tpa_dims* dims, const void* q_a, const void* q_b,
 /* Workspace bytes tpa_decode needs for these lengths (0 for invalid arguments). */
 size_t tpa_decode_workspace_bytes(const tpa_dims* dims, const int32_t* lengths, int32_t batch);
 
+/* tpa_decode without a caller-supplied workspace, for callers that cannot allocate
+ * device memory: a host application that owns every allocation and hands this
+ * library only its inputs and outputs, or a server that must not call cudaMalloc
+ * once it is running.  The paper has no counterpart; this is a deployment variant.
+ * The split-K scratch is a file-scope device array of TPA_DECODE_STATIC_SCRATCH_BYTES
+ * that every GPU loading the library holds until the process exits.  The first call
+ * on each device looks up that array's address (make it before any stream capture).
+ * Calls needing more scratch than the array holds (see tpa_decode_workspace_bytes)
+ * return TPA_ERR_WORKSPACE before any CUDA call.  All calls on a device share the
+ * array, so calls that overlap on the GPU race: keep them ordered on one stream.
+ * Nothing needs clearing between calls.  Allocates nothing.  Arguments and results
+ * are those of tpa_decode. */
+#define TPA_DECODE_STATIC_SCRATCH_BYTES (16u << 20)
+tpa_status tpa_decode_static(const tpa_dims* dims, const void* q_a, const void* q_b,
+                             const tpa_cache* cache, const int32_t* lengths, int32_t batch,
+                             void* out, tpa_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the device error word of the current
  * device.  *code receives the TPA_DEVERR_* value (NULL allowed).  Returns TPA_OK if
  * it was clear, TPA_ERR_DEVICE if a kernel recorded an error, TPA_ERR_CUDA if the

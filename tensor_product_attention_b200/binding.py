@@ -27,7 +27,9 @@ TPA_MAX_BATCH = 1024
 # Every symbol include/tpa.h declares (checked by tests/test_abi_host.py).
 EXPORTS = ("tpa_abi_version", "tpa_build_info", "tpa_status_string", "tpa_cache_bytes_per_token",
            "tpa_rope_table", "tpa_project", "tpa_cache_append", "tpa_prefill", "tpa_decode",
-           "tpa_decode_workspace_bytes", "tpa_get_device_error", "tpa_set_wait_limit")
+           "tpa_decode_workspace_bytes", "tpa_decode_static", "tpa_get_device_error",
+           "tpa_set_wait_limit")
+TPA_DECODE_STATIC_SCRATCH_BYTES = 16 << 20
 
 
 class tpa_dims(ctypes.Structure):
@@ -66,6 +68,8 @@ _sig = {
                                   _i32p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
                                   ctypes.c_size_t, ctypes.c_void_p]),
     "tpa_decode_workspace_bytes": (ctypes.c_size_t, [_P(tpa_dims), _i32p, ctypes.c_int32]),
+    "tpa_decode_static": (ctypes.c_int, [_P(tpa_dims), ctypes.c_void_p, ctypes.c_void_p, _P(tpa_cache),
+                                         _i32p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]),
     "tpa_get_device_error": (ctypes.c_int, [ctypes.c_void_p, _i32p]),
     "tpa_set_wait_limit": (None, [ctypes.c_uint32]),
 }
@@ -240,6 +244,16 @@ def tpa_decode(dims: Dims, q_a, q_b, cache: Cache, lengths, out, workspace, stre
                                          _ptr(out), _ptr(workspace),
                                          0 if workspace is None else workspace.numel() * workspace.element_size(),
                                          _stream(stream)))
+
+
+def tpa_decode_static(dims: Dims, q_a, q_b, cache: Cache, lengths, out, stream=None) -> None:
+    """tpa_decode without a workspace argument, for callers that cannot allocate device
+    memory: the scratch is the library's own fixed device array
+    (TPA_DECODE_STATIC_SCRATCH_BYTES per GPU).  Calls that overlap on the GPU race."""
+    lengths = list(lengths)
+    _check("tpa_decode_static", _lib.tpa_decode_static(ctypes.byref(dims.c()), _ptr(q_a), _ptr(q_b),
+                                                       ctypes.byref(cache.c()), _ints(lengths), len(lengths),
+                                                       _ptr(out), _stream(stream)))
 
 
 def tpa_get_device_error(stream=None) -> int:
