@@ -17,7 +17,7 @@ using namespace tpa;
 namespace {
 
 std::atomic<uint32_t> g_wait_limit{0};
-constexpr uint32_t kDefaultWaitLimit = 1u << 26;   // polls, roughly seconds of waiting
+constexpr uint32_t kDefaultWaitLimit = 1u << 24;   // polls: at most seconds of waiting
 constexpr int kMaxDevices = 64;
 std::mutex g_err_mu;
 int* g_err_ptr[kMaxDevices] = {};
