@@ -22,7 +22,9 @@
 //              a^K, a^V tiles (bulk copies) into a ring of stages
 //   warp 1     TMEM owner (512 columns) and MMA issuer; the two M-blocks ping-pong so
 //              that one block's softmax overlaps the other block's MMAs
-//   warps 2-9  softmax for M-block 0 (warps 2-5) and 1 (warps 6-9), one row per thread
+//   warps 4-11 softmax for M-block 0 (warps 4-7) and 1 (warps 8-11), one row per thread
+// The control warpgroup (warps 0-3) hands registers to the softmax warpgroups with
+// setmaxnreg once the prologue is done.
 // TMEM: U_0 [0,128), U_1 [128,256), O_0 and O_1 after 256 (d_h columns each); W_b
 // overwrites the first half of U_b once the scores are read (bf16 pairs).
 #include <algorithm>
@@ -37,7 +39,8 @@ namespace tpa {
 namespace {
 using namespace sm100;
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;   // 3 warpgroups: TMA/MMA, softmax block 0, softmax block 1
+constexpr int kRegsCtl = 96, kRegsSoftmax = 200;   // 128*96 + 256*200 = 63488 <= 384*168 (launch)
 constexpr uint32_t kBox = 128 * 128;        // one TMA box: 128 rows x 128 bytes
 constexpr float kRescale = 8.f;             // lazy rescale threshold (log2 units)
 
@@ -54,6 +57,63 @@ struct PrefillTcArgs {
     int* err;
     uint32_t wait_limit;
 };
+
+// R consecutive bf16 factor values at element offset idx*R (R = 1, 2 or 4).
+template <int R>
+__device__ __forceinline__ void load_r(const __nv_bfloat16* base, int idx, float (&f)[R]) {
+    if constexpr (R == 1) {
+        f[0] = __bfloat162float(base[idx]);
+    } else if constexpr (R == 2) {
+        const uint32_t w = reinterpret_cast<const uint32_t*>(base)[idx];
+        f[0] = bf16lo(w); f[1] = bf16hi(w);
+    } else {
+        const uint2 w = reinterpret_cast<const uint2*>(base)[idx];
+        f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+    }
+}
+
+// One pass of the softmax over a key tile for this thread's row (i, h):
+// score_j = sum_s a^K_{j,h,s} U_{(j,s)} (log2 units), mx = max_j score_j,
+// p_j = 2^(score_j - m_ref), lsum = sum_j p_j, and the W row in K order (j, s) packed
+// as bf16 pairs.  MASKED applies the causal bound j <= p_i (diagonal tiles only).
+template <int R, bool MASKED>
+__device__ __forceinline__ void softmax_pass(uint32_t u_addr, const __nv_bfloat16* ak,
+                                             const __nv_bfloat16* av, int H, int h, int j0, int p_i,
+                                             float m_ref, float& mx, float& lsum, uint32_t (&wp)[64]) {
+    constexpr int KPH = 64 / R;          // keys per 64 U columns
+    mx = -INFINITY;
+    lsum = 0.f;
+    float wprev = 0.f;
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        uint32_t u[64];
+        tmem_ld32(u_addr + (uint32_t)hf * 64u, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+        tmem_ld32(u_addr + (uint32_t)hf * 64u + 32u, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < KPH; ++q) {
+            const int jj = hf * KPH + q;
+            float fa[R], fv[R];
+            load_r<R>(ak, jj * H + h, fa);
+            float sc = 0.f;
+#pragma unroll
+            for (int sr = 0; sr < R; ++sr) sc = fmaf(fa[sr], __uint_as_float(u[q * R + sr]), sc);
+            if (MASKED) sc = (j0 + jj <= p_i) ? sc : -INFINITY;
+            mx = fmaxf(mx, sc);
+            const float p = ex2(sc - m_ref);
+            lsum += p;
+            load_r<R>(av, jj * H + h, fv);
+#pragma unroll
+            for (int sr = 0; sr < R; ++sr) {
+                float w = p * fv[sr];
+                if (MASKED) w = (p != 0.f) ? w : 0.f;
+                const int k = jj * R + sr;
+                if (k & 1) wp[k >> 1] = pack_bf16(wprev, w);
+                else wprev = w;
+            }
+        }
+    }
+}
 
 template <int DH, int R>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -114,8 +174,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     if (warp == 1) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
 
     // ---- prologue: q~ rows (bf16, 128-byte swizzled K-major) by the 256 softmax threads
-    if (warp >= 2) {
-        const int row = threadIdx.x - 64;                 // 0..255
+    if (warp >= 4) {
+        const int row = threadIdx.x - 128;                // 0..255
         const int i_loc = row / H, h = row - (row / H) * H;
         const bool vq = i_loc < nq;
         const long long t = (long long)b * a.S + q0 + (vq ? i_loc : 0);
@@ -149,8 +209,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
+    if (warp < 4) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
+      if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const uint32_t full_bytes = 2u * NB * kBox;
@@ -181,7 +242,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                         if (mbar_try_wait(&kv_full[s], (uint32_t)((fills - 1) & 1))) break;
             }
         }
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc_qk = idesc_bf16(128, UW, 0, 0);
@@ -232,9 +293,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 if (!ok) break;
             }
         }
+      }
     } else {
         // ------------------------------------------------------------ softmax
-        const int bl = (warp - 2) >> 2;
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+        const int bl = (warp - 4) >> 2;
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;                 // TMEM lane
         const int row = bl * 128 + r;
@@ -246,6 +309,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         const uint32_t o_col = 256u + (uint32_t)bl * DH;
         float m_use = -INFINITY, l = 0.f;
         bool alive = true;
+        const uint32_t u_addr = lane_addr + u_col;
         for (int t = 0; t < n_tiles; ++t) {
             if (!mbar_wait(&u_ready[bl], (uint32_t)(t & 1), lim, a.err, abort)) { alive = false; break; }
             tc_fence_after();
@@ -253,85 +317,59 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             const int j0 = t * KT;
             const __nv_bfloat16* ak = stage_ak(s);
             const __nv_bfloat16* av = stage_av(s);
-            float sc[KT];
-#pragma unroll
-            for (int c = 0; c < UW / 32; ++c) {
-                uint32_t u[32];
-                tmem_ld32(lane_addr + u_col + (uint32_t)c * 32u, u);
-                tmem_ld_wait();
-#pragma unroll
-                for (int q = 0; q < 32 / R; ++q) {
-                    const int jj = c * (32 / R) + q;
-                    float v = 0.f;
-#pragma unroll
-                    for (int sr = 0; sr < R; ++sr)
-                        v = fmaf(__bfloat162float(ak[(jj * H + h) * R + sr]), __uint_as_float(u[q * R + sr]), v);
-                    sc[jj] = (j0 + jj <= p_i) ? v : -INFINITY;
+            const bool masked = j0 + KT - 1 > p0;        // same for every row of the CTA
+            uint32_t wp[64];
+            float mx = -INFINITY, lsum = 0.f;
+            bool ok = false;
+            if (t > 0) {
+                // common case: one pass against the running max
+                if (masked) softmax_pass<R, true>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
+                else softmax_pass<R, false>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
+                ok = mx <= m_use + kRescale;
+            }
+            if (__all_sync(0xffffffffu, ok)) {
+                l += lsum;
+            } else {
+                // first tile, or the max rose by more than 2^kRescale: exact max, rescale O
+                if (t == 0) {
+                    if (masked) softmax_pass<R, true>(u_addr, ak, av, H, h, j0, p_i, INFINITY, mx, lsum, wp);
+                    else softmax_pass<R, false>(u_addr, ak, av, H, h, j0, p_i, INFINITY, mx, lsum, wp);
                 }
-            }
-            float m_t = -INFINITY;
+                const float m_new = (t == 0 || mx > m_use + kRescale) ? mx : m_use;
+                const float alpha = (t == 0) ? 1.f : ex2(m_use - m_new);
+                if (t > 0) l *= alpha;
+                if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    // O row *= alpha (PV(t-1) has completed: QK(t) was committed after it)
 #pragma unroll
-            for (int jj = 0; jj < KT; ++jj) m_t = fmaxf(m_t, sc[jj]);
-            float alpha = 1.f;
-            bool resc = false;
-            if (t == 0) {
-                m_use = m_t;
-            } else if (m_t > m_use + kRescale) {
-                alpha = exp2f(m_use - m_t);
-                m_use = m_t;
-                l *= alpha;
-                resc = true;
-            }
-            if (__any_sync(0xffffffffu, resc)) {
-                // O row *= alpha (PV(t-1) has completed: QK(t) was committed after it)
+                    for (int c = 0; c < DH / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(lane_addr + o_col + (uint32_t)c * 32u, o);
+                        tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < DH / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(lane_addr + o_col + (uint32_t)c * 32u, o);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st32(lane_addr + o_col + (uint32_t)c * 32u, o);
-                }
-                tmem_st_wait();
-            }
-            // p = exp2(score - m) once per key (0 for masked keys), row sum l
-#pragma unroll
-            for (int jj = 0; jj < KT; ++jj) {
-                const float p = exp2f(sc[jj] - m_use);
-                sc[jj] = p;
-                l += p;
-            }
-            // W = p * a^V as bf16 pairs in K order (j, s), written over U's first half;
-            // masked keys give exactly 0 whatever the cache holds past the valid length
-#pragma unroll
-            for (int c = 0; c < UW / 64; ++c) {
-                uint32_t wp[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float wv[2];
-#pragma unroll
-                    for (int hl = 0; hl < 2; ++hl) {
-                        const int kidx = c * 64 + 2 * e + hl;        // K index = jj*R + sr
-                        const int jj = kidx / R, sr = kidx % R;
-                        const float p = sc[jj];
-                        wv[hl] = p != 0.f ? p * __bfloat162float(av[(jj * H + h) * R + sr]) : 0.f;
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(lane_addr + o_col + (uint32_t)c * 32u, o);
                     }
-                    wp[e] = pack_bf16(wv[0], wv[1]);
+                    tmem_st_wait();
                 }
-                tmem_st32(lane_addr + u_col + (uint32_t)c * 32u, wp);
+                m_use = m_new;
+                if (masked) softmax_pass<R, true>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
+                else softmax_pass<R, false>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
+                l += lsum;
             }
+            // W over the first half of U (the scores have all been read)
+            tmem_st32(u_addr, *reinterpret_cast<uint32_t(*)[32]>(&wp[0]));
+            tmem_st32(u_addr + 32u, *reinterpret_cast<uint32_t(*)[32]>(&wp[32]));
             tmem_st_wait();
             if (bl == 0 && t == n_tiles - 1 && j0 + KT > kv_len) {
                 // keys at or past the valid length: clear their b^V rows so that
                 // 0 * (whatever the cache holds there) stays 0 in the PV product
                 uint8_t* bv = stage_bv(s);
                 const int first = (kv_len - j0) * R;
-                for (int rr = first + (threadIdx.x - 64); rr < 128; rr += 128)
+                for (int rr = first + (threadIdx.x - 128); rr < 128; rr += 128)
                     for (int cb = 0; cb < NB; ++cb) {
-                        uint4* p = reinterpret_cast<uint4*>(bv + cb * kBox + rr * 128);
+                        uint4* pz = reinterpret_cast<uint4*>(bv + cb * kBox + rr * 128);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) p[e] = make_uint4(0, 0, 0, 0);
+                        for (int e = 0; e < 8; ++e) pz[e] = make_uint4(0, 0, 0, 0);
                     }
                 fence_proxy_async_smem();
             }

@@ -263,6 +263,16 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t byte_in_
     return row * 128u + (chunk << 4) + (byte_in_row & 15u);
 }
 
+// 2^x on the MUFU unit (approximate, flushes denormals; 2^-inf = +0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
