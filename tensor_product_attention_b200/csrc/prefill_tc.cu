@@ -72,17 +72,57 @@ __device__ __forceinline__ void load_r(const __nv_bfloat16* base, int idx, float
     }
 }
 
-// One pass of the softmax over a key tile for this thread's row (i, h):
-// score_j = sum_s a^K_{j,h,s} U_{(j,s)} (log2 units), mx = max_j score_j,
-// p_j = 2^(score_j - m_ref), lsum = sum_j p_j, and the W row in K order (j, s) packed
-// as bf16 pairs.  MASKED applies the causal bound j <= p_i (diagonal tiles only).
-template <int R, bool MASKED>
+// One pass of the softmax over a key tile for this thread's row (i, h), relative to a
+// reference max m_ref: d_j = sum_s a^K_{j,h,s} U_{(j,s)} - m_ref (log2 units), mx =
+// max_j d_j, p_j = 2^d_j, lsum = sum_j p_j, and the W row (p_j a^V_{j,h,s}) in K order
+// (j, s) packed as bf16 pairs.  MASKED applies the causal bound j <= p_i (diagonal tiles).
+template <int R, bool MASKED, int HS_>
 __device__ __forceinline__ void softmax_pass(uint32_t u_addr, const __nv_bfloat16* ak,
                                              const __nv_bfloat16* av, int H, int h, int j0, int p_i,
                                              float m_ref, float& mx, float& lsum, uint32_t (&wp)[64]) {
-    constexpr int KPH = 64 / R;          // keys per 64 U columns
+    const int HS = HS_ > 0 ? HS_ : H;   // head count, compile-time when known
     mx = -INFINITY;
     lsum = 0.f;
+    if constexpr (R == 2) {
+        // one 32-bit word holds a key's two factor values; W = bf16x2(p) * (a^V pair).
+        // Four independent max/sum accumulators keep the loop-carried chains short.
+        const uint32_t* akr = reinterpret_cast<const uint32_t*>(ak) + h;
+        const uint32_t* avr = reinterpret_cast<const uint32_t*>(av) + h;
+        float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float lsa[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            uint32_t u[64];
+            tmem_ld32(u_addr + (uint32_t)hf * 64u, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+            tmem_ld32(u_addr + (uint32_t)hf * 64u + 32u, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+            uint32_t wa[32], wv[32];
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                wa[q] = akr[(hf * 32 + q) * HS];
+                wv[q] = avr[(hf * 32 + q) * HS];
+            }
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const int jj = hf * 32 + q;
+                float d = fmaf(bf16lo(wa[q]), __uint_as_float(u[2 * q]), -m_ref);
+                d = fmaf(bf16hi(wa[q]), __uint_as_float(u[2 * q + 1]), d);
+                if (MASKED) d = (j0 + jj <= p_i) ? d : -INFINITY;
+                mxa[q & 3] = fmaxf(mxa[q & 3], d);
+                const float p = ex2(d);
+                lsa[q & 3] += p;
+                const __nv_bfloat162 pw = __float2bfloat162_rn(p);
+                const __nv_bfloat162 prod = __hmul2(pw, *reinterpret_cast<const __nv_bfloat162*>(&wv[q]));
+                uint32_t w = *reinterpret_cast<const uint32_t*>(&prod);
+                if (MASKED) w = (p != 0.f) ? w : 0u;
+                wp[jj] = w;
+            }
+        }
+        mx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
+        lsum = (lsa[0] + lsa[1]) + (lsa[2] + lsa[3]);
+        return;
+    }
+    constexpr int KPH = 64 / R;          // keys per 64 U columns
     float wprev = 0.f;
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
@@ -94,15 +134,15 @@ __device__ __forceinline__ void softmax_pass(uint32_t u_addr, const __nv_bfloat1
         for (int q = 0; q < KPH; ++q) {
             const int jj = hf * KPH + q;
             float fa[R], fv[R];
-            load_r<R>(ak, jj * H + h, fa);
-            float sc = 0.f;
+            load_r<R>(ak, jj * HS + h, fa);
+            float d = -m_ref;
 #pragma unroll
-            for (int sr = 0; sr < R; ++sr) sc = fmaf(fa[sr], __uint_as_float(u[q * R + sr]), sc);
-            if (MASKED) sc = (j0 + jj <= p_i) ? sc : -INFINITY;
-            mx = fmaxf(mx, sc);
-            const float p = ex2(sc - m_ref);
+            for (int sr = 0; sr < R; ++sr) d = fmaf(fa[sr], __uint_as_float(u[q * R + sr]), d);
+            if (MASKED) d = (j0 + jj <= p_i) ? d : -INFINITY;
+            mx = fmaxf(mx, d);
+            const float p = ex2(d);
             lsum += p;
-            load_r<R>(av, jj * H + h, fv);
+            load_r<R>(av, jj * HS + h, fv);
 #pragma unroll
             for (int sr = 0; sr < R; ++sr) {
                 float w = p * fv[sr];
@@ -115,7 +155,7 @@ __device__ __forceinline__ void softmax_pass(uint32_t u_addr, const __nv_bfloat1
     }
 }
 
-template <int DH, int R>
+template <int DH, int R, int HC>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                   const PrefillTcArgs a, const SeqParams start) {
@@ -139,7 +179,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int H = a.H;
+    const int H = HC > 0 ? HC : a.H;
     const int qb = a.n_qblocks - 1 - (int)blockIdx.x;   // longest rows first
     const int b = blockIdx.y;
     const int q0 = qb * a.qpb;
@@ -323,19 +363,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             bool ok = false;
             if (t > 0) {
                 // common case: one pass against the running max
-                if (masked) softmax_pass<R, true>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
-                else softmax_pass<R, false>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
-                ok = mx <= m_use + kRescale;
+                if (masked) softmax_pass<R, true, HC>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
+                else softmax_pass<R, false, HC>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
+                ok = mx <= kRescale;
             }
             if (__all_sync(0xffffffffu, ok)) {
                 l += lsum;
             } else {
                 // first tile, or the max rose by more than 2^kRescale: exact max, rescale O
                 if (t == 0) {
-                    if (masked) softmax_pass<R, true>(u_addr, ak, av, H, h, j0, p_i, INFINITY, mx, lsum, wp);
-                    else softmax_pass<R, false>(u_addr, ak, av, H, h, j0, p_i, INFINITY, mx, lsum, wp);
+                    if (masked) softmax_pass<R, true, HC>(u_addr, ak, av, H, h, j0, p_i, 0.f, mx, lsum, wp);
+                    else softmax_pass<R, false, HC>(u_addr, ak, av, H, h, j0, p_i, 0.f, mx, lsum, wp);
                 }
-                const float m_new = (t == 0 || mx > m_use + kRescale) ? mx : m_use;
+                const float m_new = (t == 0) ? mx : (mx > kRescale ? m_use + mx : m_use);
                 const float alpha = (t == 0) ? 1.f : ex2(m_use - m_new);
                 if (t > 0) l *= alpha;
                 if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -352,8 +392,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     tmem_st_wait();
                 }
                 m_use = m_new;
-                if (masked) softmax_pass<R, true>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
-                else softmax_pass<R, false>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
+                if (masked) softmax_pass<R, true, HC>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
+                else softmax_pass<R, false, HC>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
                 l += lsum;
             }
             // W over the first half of U (the scores have all been read)
@@ -408,7 +448,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     }
 }
 
-template <int DH, int R>
+template <int DH, int R, int HC>
 cudaError_t launch_t(const PrefillTcArgs& a0, const tpa_cache& c, int batch, const SeqParams& start,
                      cudaStream_t st) {
     PrefillTcArgs a = a0;
@@ -428,11 +468,11 @@ cudaError_t launch_t(const PrefillTcArgs& a0, const tpa_cache& c, int batch, con
     if (!make_tmap_bf16(&tmk, c.b_k, 2, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 2, dims, stride, box))
         return cudaErrorInvalidValue;
     const size_t smem = 1024 + q_bytes + (size_t)a.stages * a.stage_bytes + (2 * a.stages + 6) * 8 + 16;
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<DH, R>,
+    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<DH, R, HC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.n_qblocks, batch);
-    prefill_tc_kernel<DH, R><<<grid, kThreads, smem, st>>>(tmk, tmv, a, start);
+    prefill_tc_kernel<DH, R, HC><<<grid, kThreads, smem, st>>>(tmk, tmv, a, start);
     return cudaGetLastError();
 }
 }  // namespace
@@ -467,14 +507,17 @@ cudaError_t launch_prefill_tc(const Shape& s, const tpa_factors& q, const tpa_ca
     a.out_scale = 1.f / (float)s.Rv;
     a.err = err;
     a.wait_limit = wait_limit;
+    // head count 16 gets constant strides in the softmax loop; others read it at run time
     if (s.Dh == 64) {
-        if (s.Rk == 1) return launch_t<64, 1>(a, c, batch, start, st);
-        if (s.Rk == 2) return launch_t<64, 2>(a, c, batch, start, st);
-        return launch_t<64, 4>(a, c, batch, start, st);
+        if (s.Rk == 2) return s.H == 16 ? launch_t<64, 2, 16>(a, c, batch, start, st)
+                                        : launch_t<64, 2, 0>(a, c, batch, start, st);
+        if (s.Rk == 1) return launch_t<64, 1, 0>(a, c, batch, start, st);
+        return launch_t<64, 4, 0>(a, c, batch, start, st);
     }
-    if (s.Rk == 1) return launch_t<128, 1>(a, c, batch, start, st);
-    if (s.Rk == 2) return launch_t<128, 2>(a, c, batch, start, st);
-    return launch_t<128, 4>(a, c, batch, start, st);
+    if (s.Rk == 2) return s.H == 16 ? launch_t<128, 2, 16>(a, c, batch, start, st)
+                                    : launch_t<128, 2, 0>(a, c, batch, start, st);
+    if (s.Rk == 1) return launch_t<128, 1, 0>(a, c, batch, start, st);
+    return launch_t<128, 4, 0>(a, c, batch, start, st);
 }
 
 }  // namespace tpa
