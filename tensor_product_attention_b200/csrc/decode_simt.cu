@@ -16,29 +16,74 @@
 
 #include "tpa_internal.h"
 #include "device_util.cuh"
+#include "tmap.h"
 
 namespace tpa {
 
-DecodeSchedule decode_schedule(const Shape& s, const int32_t* lengths, int batch) {
+void make_decode_plan(const Shape& s, const int32_t* lengths, int batch, bool tc,
+                      DecodePlan* plan) {
+    DecodePlan& P = *plan;
+    P.batch = batch;
     long long total = 0;
-    int max_len = 1;
     for (int b = 0; b < batch; ++b) {
+        P.len[b] = lengths[b];
         total += lengths[b];
-        max_len = std::max(max_len, (int)lengths[b]);
     }
-    const int tile = 128;
-    const long long target_ctas = 148LL * 4;
-    long long per = (total + target_ctas - 1) / target_ctas;
-    int split_len = (int)std::max<long long>(tile, ((per + tile - 1) / tile) * tile);
-    DecodeSchedule sch;
-    sch.split_len = split_len;
-    sch.max_splits = (max_len + split_len - 1) / split_len;
-    return sch;
+    if (!tc) {
+        // splits of split_len keys (a multiple of 128), about 4 CTAs per SM in all
+        const int tile = 128;
+        const long long target_ctas = (long long)sm_count() * 4;
+        const long long per = (total + target_ctas - 1) / target_ctas;
+        P.split_len = (int)std::max<long long>(tile, ((per + tile - 1) / tile) * tile);
+        P.key_tile = tile;
+        int part = 0, max_splits = 1;
+        for (int b = 0; b < batch; ++b) {
+            P.first_part[b] = part;
+            P.n_parts[b] = (lengths[b] + P.split_len - 1) / P.split_len;
+            part += P.n_parts[b];
+            max_splits = std::max(max_splits, (int)P.n_parts[b]);
+        }
+        P.total_parts = part;
+        P.n_ctas = max_splits;          // grid.x of the split kernel
+        P.total_tiles = 0;
+        return;
+    }
+    // persistent grid over the concatenated key tiles of all sequences
+    const int kt = 128 / s.Rk;
+    P.key_tile = kt;
+    P.split_len = 0;
+    long long n = 0;
+    for (int b = 0; b < batch; ++b) {
+        P.tile_prefix[b] = (int32_t)n;
+        n += (lengths[b] + kt - 1) / kt;
+    }
+    P.tile_prefix[batch] = (int32_t)n;
+    P.total_tiles = (int32_t)n;
+    const int G = (int)std::min<long long>(sm_count(), n);
+    P.n_ctas = G;
+    auto g0 = [&](long long c) { return c * n / G; };
+    // parts in (CTA, sequence) order; the parts of one sequence are consecutive
+    int part = 0;
+    int b = 0;
+    for (int b2 = 0; b2 < batch; ++b2) P.n_parts[b2] = 0;
+    for (int c = 0; c < G; ++c) {
+        const long long lo = g0(c), hi = g0(c + 1);
+        while (b < batch && P.tile_prefix[b + 1] <= lo) ++b;
+        for (int bb = b; bb < batch && P.tile_prefix[bb] < hi; ++bb) {
+            if (P.tile_prefix[bb + 1] <= lo) continue;
+            if (P.n_parts[bb] == 0) {
+                P.first_part[bb] = part;
+                P.c_first[bb] = c;
+            }
+            ++P.n_parts[bb];
+            ++part;
+        }
+    }
+    P.total_parts = part;
 }
 
-size_t decode_workspace_bytes(const Shape& s, const DecodeSchedule& sch, int batch) {
-    size_t parts = (size_t)batch * sch.max_splits * s.H;
-    return parts * (2 + (size_t)s.Dh) * sizeof(float);
+size_t decode_workspace_bytes(const Shape& s, const DecodePlan& plan) {
+    return (size_t)plan.total_parts * s.H * (2 + (size_t)s.Dh) * sizeof(float);
 }
 
 namespace {
@@ -49,15 +94,15 @@ constexpr int MAXO = 32;   // output elements per thread: h*d_h <= 8192
 struct DecodeArgs {
     const void *q_a, *q_b;
     const void *ca_k, *ca_v, *cb_k, *cb_v;
-    float* ws_ml;   // [batch][max_splits][H][2]
-    float* ws_o;    // [batch][max_splits][H][Dh]
-    int H, Dh, Rq, Rk, Rv, cap, split_len, max_splits;
+    float* ws_ml;   // [parts][H][2]
+    float* ws_o;    // [parts][H][Dh]
+    int H, Dh, Rq, Rk, Rv, cap, split_len;
 };
 
 template <typename T>
-__global__ void __launch_bounds__(NT) decode_simt_kernel(DecodeArgs a, SeqParams len) {
+__global__ void __launch_bounds__(NT) decode_simt_kernel(DecodeArgs a, const DecodePlan plan) {
     const int split = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-    const int L = len.v[b];
+    const int L = plan.len[b];
     const int j0 = split * a.split_len;
     if (j0 >= L) return;
     const int j1 = min(L, j0 + a.split_len);
@@ -171,7 +216,7 @@ __global__ void __launch_bounds__(NT) decode_simt_kernel(DecodeArgs a, SeqParams
         }
     }
     __syncthreads();
-    const long long part = ((long long)b * a.max_splits + split) * H;
+    const long long part = (long long)(plan.first_part[b] + split) * H;
     for (int h = tid; h < H; h += NT) {
         a.ws_ml[(part + h) * 2 + 0] = mrow[h];
         a.ws_ml[(part + h) * 2 + 1] = lrow[h];
@@ -187,15 +232,16 @@ struct CombineArgs {
     const float* ws_ml;
     const float* ws_o;
     void* out;
-    int H, Dh, Rv, split_len, max_splits;
+    int H, Dh, Rv;
 };
 
-// grid (H, batch), one thread per output element of the head.
+// grid (H, batch), one thread per output element of the head.  Parts are merged in
+// increasing part order, so the result does not depend on scheduling.
 template <typename T>
-__global__ void decode_combine_kernel(CombineArgs a, SeqParams len) {
+__global__ void decode_combine_kernel(CombineArgs a, const DecodePlan plan) {
     const int h = blockIdx.x, b = blockIdx.y;
-    const int nsplit = (len.v[b] + a.split_len - 1) / a.split_len;
-    const long long base = (long long)b * a.max_splits;
+    const int nsplit = plan.n_parts[b];
+    const long long base = plan.first_part[b];
     float m = -INFINITY;
     for (int k = 0; k < nsplit; ++k) m = fmaxf(m, a.ws_ml[((base + k) * a.H + h) * 2]);
     float den = 0.f;
@@ -224,49 +270,47 @@ static size_t decode_simt_smem(const Shape& s) {
 }
 
 cudaError_t launch_decode_simt(const Shape& s, const void* q_a, const void* q_b,
-                               const tpa_cache& c, const SeqParams& len, int batch,
-                               const DecodeSchedule& sch, float* ws, cudaStream_t st) {
+                               const tpa_cache& c, const DecodePlan& plan, float* ws,
+                               cudaStream_t st) {
     if ((long long)s.H * s.Dh > (long long)NT * MAXO) return cudaErrorInvalidValue;
     DecodeArgs a;
     a.q_a = q_a; a.q_b = q_b;
     a.ca_k = c.a_k; a.ca_v = c.a_v; a.cb_k = c.b_k; a.cb_v = c.b_v;
     a.ws_ml = ws;
-    a.ws_o = ws + (size_t)batch * sch.max_splits * s.H * 2;
+    a.ws_o = ws + (size_t)plan.total_parts * s.H * 2;
     a.H = s.H; a.Dh = s.Dh; a.Rq = s.Rq; a.Rk = s.Rk; a.Rv = s.Rv; a.cap = c.capacity;
-    a.split_len = sch.split_len; a.max_splits = sch.max_splits;
+    a.split_len = plan.split_len;
     size_t smem = decode_simt_smem(s);
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
-    dim3 grid(sch.max_splits, batch);
+    dim3 grid(plan.n_ctas, plan.batch);
     cudaError_t e;
     if (s.bf16) {
         e = cudaFuncSetAttribute(decode_simt_kernel<__nv_bfloat16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        decode_simt_kernel<__nv_bfloat16><<<grid, NT, smem, st>>>(a, len);
+        decode_simt_kernel<__nv_bfloat16><<<grid, NT, smem, st>>>(a, plan);
     } else {
         e = cudaFuncSetAttribute(decode_simt_kernel<float>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        decode_simt_kernel<float><<<grid, NT, smem, st>>>(a, len);
+        decode_simt_kernel<float><<<grid, NT, smem, st>>>(a, plan);
     }
     return cudaGetLastError();
 }
 
-cudaError_t launch_decode_combine(const Shape& s, const SeqParams& len, int batch,
-                                  const DecodeSchedule& sch, const float* ws, void* out,
-                                  cudaStream_t st) {
+cudaError_t launch_decode_combine(const Shape& s, const DecodePlan& plan, const float* ws,
+                                  void* out, cudaStream_t st) {
     CombineArgs a;
     a.ws_ml = ws;
-    a.ws_o = ws + (size_t)batch * sch.max_splits * s.H * 2;
+    a.ws_o = ws + (size_t)plan.total_parts * s.H * 2;
     a.out = out;
-    a.H = s.H; a.Dh = s.Dh; a.Rv = s.Rv; a.split_len = sch.split_len;
-    a.max_splits = sch.max_splits;
-    dim3 grid(s.H, batch);
+    a.H = s.H; a.Dh = s.Dh; a.Rv = s.Rv;
+    dim3 grid(s.H, plan.batch);
     int threads = std::min(256, ((s.Dh + 31) / 32) * 32);
     if (s.bf16)
-        decode_combine_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(a, len);
+        decode_combine_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(a, plan);
     else
-        decode_combine_kernel<float><<<grid, threads, 0, st>>>(a, len);
+        decode_combine_kernel<float><<<grid, threads, 0, st>>>(a, plan);
     return cudaGetLastError();
 }
 

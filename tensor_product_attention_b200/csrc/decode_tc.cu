@@ -1,10 +1,490 @@
-// Decode on tcgen05 tensor cores (placeholder until the kernel lands).
+// Decode from the factor cache on tcgen05 tensor cores (bf16, fp32 accumulate).
+//
+// One query per sequence at position len-1 attends to the cached keys 0..len-1
+// ("【拜读】Tensor Product Attention Is All You Need…" (coreui.cn), 代码 前向传播: the
+// cache is written, then read over [:start_pos+seqlen]), reading only the factors; B_K
+// is used as cached, already rotated (same page, 关键问题及回答 问题2).  With the query
+// folded once per sequence, q~_h = log2(e)/(R_Q R_K sqrt(d_h)) sum_r a^Q_{h,r} b^Q_r
+// (or the given per-head q for TPA-KVonly), a tile of KT = 128/R keys costs:
+//   U^T  = b^K . q~^T     tcgen05, M = 128 rows (key j, rank s), N = h, K = d_h
+//   score_h(j) = sum_s a^K_{j,h,s} U^T_{(j,s),h}      one thread per row, shfl over s
+//   W^T_{(j,s),h} = 2^(score - m_h) a^V_{j,h,s}        bf16, to shared memory
+//   O^T += b^V^T . W^T    tcgen05, M = d_h (A = b^V tile read MN-major), N = h, K = 128
+// HBM-bound: only (R_K + R_V)(h + d_h) factor elements per key are read.
+//
+// Scheduling: a persistent grid of one CTA per SM walks the key tiles of all
+// sequences concatenated; CTA c takes tiles [c*N/G, (c+1)*N/G), so ragged lengths are
+// balanced exactly.  Each (CTA, sequence) overlap ("part") writes its partial softmax
+// state (m_h, l_h, O^T) to the workspace; the combine kernel merges the parts of a
+// sequence in a fixed order.  The softmax keeps a CTA-wide reference max per head and
+// only revisits it (rescaling O^T in tensor memory) when a score exceeds it by more
+// than 2^8, so a tile normally needs one pass and one barrier.
+//
+// Warp roles: warp 0 TMA (two stages of b^K/b^V tiles, 128-byte swizzle, and a^K/a^V
+// bulk copies), warp 1 TMEM owner and MMA issuer, warps 2.. softmax (4 warps per 16
+// heads; TMEM lane = row).  TMEM: U^T double-buffered (2 x h columns) and O^T (h).
+#include <algorithm>
+#include <cmath>
+
 #include "tpa_internal.h"
+#include "sm100.cuh"
+#include "tmap.h"
+
 namespace tpa {
-bool decode_tc_supported(const Shape&) { return false; }
-cudaError_t launch_decode_tc(const Shape&, const void*, const void*, const tpa_cache&,
-                             const SeqParams&, int, const DecodeSchedule&, float*, int*, uint32_t,
-                             cudaStream_t) {
-    return cudaErrorNotSupported;
+
+namespace {
+using namespace sm100;
+
+constexpr int DH = 128;                  // head dim (M of the value MMA)
+constexpr uint32_t kBox = 128 * 128;     // one TMA box: 128 rows x 128 bytes
+constexpr float kTau = 8.f;              // lazy rescale threshold (log2 units)
+constexpr int kStages = 2;
+
+struct DecodeTcArgs {
+    const __nv_bfloat16* q_a;      // [B][H][Rq] or null
+    const __nv_bfloat16* q_b;      // [B][Rq][DH] or q [B][H][DH]
+    const __nv_bfloat16* ca_k;     // [B][cap][H][R]
+    const __nv_bfloat16* ca_v;
+    float* ws_ml;                  // [parts][H][2]
+    float* ws_o;                   // [parts][H][DH]
+    int Rq, cap;
+    float qscale;
+    uint32_t a_bytes, stage_bytes;
+    int* err;
+    uint32_t wait_limit;
+};
+
+// tile bookkeeping shared by every role: which sequence / local tile a CTA tile is
+template <int KT>
+struct TileWalk {
+    int b;           // current sequence
+    __device__ void init(const DecodePlan& P, int g) {
+        b = 0;
+        while (P.tile_prefix[b + 1] <= g) ++b;
+    }
+    __device__ void advance(const DecodePlan& P, int g) {
+        while (P.tile_prefix[b + 1] <= g) ++b;
+    }
+};
+
+template <int HH, int R>
+__global__ void __launch_bounds__(64 + 32 * 4 * (HH / 16), 1)
+decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                 const DecodeTcArgs a, const DecodePlan P) {
+    constexpr int KT = 128 / R;                 // keys per tile
+    constexpr int NG = HH / 16;                 // head groups of 16 (4 warps each)
+    constexpr int NSM = 128 * NG;               // softmax threads
+    constexpr uint32_t kQW = HH * 256u;         // q~ or W^T buffer: 2 x [HH rows][128 B]
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* stg = smem;                                            // kStages stages
+    uint8_t* qbuf = stg + (size_t)kStages * a.stage_bytes;          // 2 x q~
+    uint8_t* wbuf = qbuf + 2 * kQW;                                 // 2 x W^T
+    float* red = reinterpret_cast<float*>(wbuf + 2 * kQW);          // [NG][4][16] scratch
+    uint64_t* bars = reinterpret_cast<uint64_t*>(red + NG * 64);
+    uint64_t* kv_full = bars;                    // [kStages]
+    uint64_t* kv_empty = kv_full + kStages;      // [kStages]
+    uint64_t* u_full = kv_empty + kStages;       // [2]
+    uint64_t* w_full = u_full + 2;               // [2]
+    uint64_t* w_empty = w_full + 2;              // [2]
+    uint64_t* q_ready = w_empty + 2;             // [2]
+    uint64_t* o_done = q_ready + 2;              // [1]
+    uint64_t* o_free = o_done + 1;               // [1]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 1);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    auto st_bk = [&](int s) { return stg + (size_t)s * a.stage_bytes; };
+    auto st_bv = [&](int s) { return stg + (size_t)s * a.stage_bytes + 2 * kBox; };
+    auto st_ak = [&](int s) { return stg + (size_t)s * a.stage_bytes + 4 * kBox; };
+    auto st_av = [&](int s) {
+        return stg + (size_t)s * a.stage_bytes + 4 * kBox + ((a.a_bytes + 127u) & ~127u);
+    };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x;
+    const long long N = P.total_tiles, G = gridDim.x;
+    const int g0 = (int)(c * N / G), g1 = (int)((c + 1) * N / G);
+    const int n = g1 - g0;
+    const uint32_t lim = a.wait_limit;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&u_full[i], 1);
+            mbar_init(&w_full[i], NSM);
+            mbar_init(&w_empty[i], 1);
+            mbar_init(&q_ready[i], 1);
+        }
+        mbar_init(o_done, 1);
+        mbar_init(o_free, NSM);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) { prefetch_tensormap(&tmk); prefetch_tensormap(&tmv); }
+    if (warp == 1) { tmem_alloc(tmem_slot, 128); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0 && n > 0) {
+            TileWalk<KT> tw;
+            tw.init(P, g0);
+            int i = 0;
+            for (; i < n && !*abort; ++i) {
+                const int g = g0 + i;
+                tw.advance(P, g);
+                const int b = tw.b;
+                const int j0 = (g - P.tile_prefix[b]) * KT;
+                const int s = i % kStages;
+                if (i >= kStages &&
+                    !mbar_wait(&kv_empty[s], (uint32_t)((i / kStages - 1) & 1), lim, a.err, abort))
+                    break;
+                const int rows_a = min(KT, a.cap - j0);
+                const uint32_t abytes = (uint32_t)rows_a * HH * R * 2u;
+                mbar_arrive_expect_tx(&kv_full[s], 4u * kBox + 2u * abytes);
+                const int y = (int)(((long long)b * a.cap + j0) * R);
+                tma_load_2d(st_bk(s), &tmk, &kv_full[s], 0, y);
+                tma_load_2d(st_bk(s) + kBox, &tmk, &kv_full[s], 64, y);
+                tma_load_2d(st_bv(s), &tmv, &kv_full[s], 0, y);
+                tma_load_2d(st_bv(s) + kBox, &tmv, &kv_full[s], 64, y);
+                const long long ea = ((long long)b * a.cap + j0) * HH * R;
+                bulk_load(st_ak(s), a.ca_k + ea, abytes, &kv_full[s]);
+                bulk_load(st_av(s), a.ca_v + ea, abytes, &kv_full[s]);
+            }
+            for (int s = 0; s < kStages; ++s) {                 // drain issued copies
+                const int fills = i > s ? (i - s - 1) / kStages + 1 : 0;
+                if (fills > 0)
+                    for (uint32_t k = 0; k < lim; ++k)
+                        if (mbar_try_wait(&kv_full[s], (uint32_t)((fills - 1) & 1))) break;
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0 && n > 0) {
+            const uint32_t idesc_qk = idesc_bf16(128, HH, 0, 0);
+            const uint32_t idesc_pv = idesc_bf16(128, HH, 1, 0);
+            const uint32_t q0 = smem_u32(qbuf), w0 = smem_u32(wbuf);
+            TileWalk<KT> twq, twp;
+            twq.init(P, g0);
+            twp.init(P, g0);
+            int segq = -1, segp = -1;     // segment counters for the QK and PV streams
+            int prev_bq = -1, prev_bp = -1;
+            // PV(j) for the previous tile; returns false on a failed wait
+            auto issue_pv = [&](int j) -> bool {
+                const int g = g0 + j;
+                twp.advance(P, g);
+                const bool first = twp.b != prev_bp;
+                if (first) { ++segp; prev_bp = twp.b; }
+                const bool last = (j == n - 1) || (P.tile_prefix[twp.b + 1] <= g + 1);
+                if (!mbar_wait(&w_full[j & 1], (uint32_t)((j >> 1) & 1), lim, a.err, abort)) return false;
+                if (first && segp > 0 &&
+                    !mbar_wait(o_free, (uint32_t)((segp - 1) & 1), lim, a.err, abort))
+                    return false;
+                tc_fence_after();
+                const int s = j % kStages;
+                const uint32_t bv = smem_u32(st_bv(s));
+                const uint32_t wb = w0 + (uint32_t)(j & 1) * kQW;
+#pragma unroll
+                for (int k = 0; k < 128 / 16; ++k) {
+                    mma_ss(tmem + 2u * HH, smem_desc(bv + (uint32_t)k * 2048u, kBox, 1024, kSwizzle128),
+                           smem_desc(wb + (uint32_t)(k >> 2) * (HH * 128u) + (uint32_t)(k & 3) * 32u,
+                                     16, 1024, kSwizzle128),
+                           idesc_pv, (first && k == 0) ? 0u : 1u);
+                }
+                mma_commit(&w_empty[j & 1]);
+                mma_commit(&kv_empty[s]);
+                if (last) mma_commit(o_done);
+                return true;
+            };
+            for (int i = 0; i <= n && !*abort; ++i) {
+                bool newseg = false;
+                if (i < n) {
+                    twq.advance(P, g0 + i);
+                    newseg = twq.b != prev_bq;
+                }
+                // At a sequence boundary the previous part's last PV goes first: the
+                // softmax reads that part's O^T before it builds the next q~.
+                const bool pv_first = i >= 1 && (i == n || newseg);
+                if (pv_first && !issue_pv(i - 1)) break;
+                if (i < n) {
+                    if (newseg) {
+                        ++segq;
+                        prev_bq = twq.b;
+                        if (!mbar_wait(&q_ready[segq & 1], (uint32_t)((segq >> 1) & 1), lim, a.err, abort)) break;
+                    }
+                    const int s = i % kStages;
+                    if (!mbar_wait(&kv_full[s], (uint32_t)((i / kStages) & 1), lim, a.err, abort)) break;
+                    tc_fence_after();
+                    const uint32_t bk = smem_u32(st_bk(s));
+                    const uint32_t qb = q0 + (uint32_t)(segq & 1) * kQW;
+#pragma unroll
+                    for (int k = 0; k < DH / 16; ++k) {
+                        const uint32_t cb = (uint32_t)(k >> 2), kk = (uint32_t)(k & 3) * 32u;
+                        mma_ss(tmem + (uint32_t)(i & 1) * HH,
+                               smem_desc(bk + cb * kBox + kk, 16, 1024, kSwizzle128),
+                               smem_desc(qb + cb * (HH * 128u) + kk, 16, 1024, kSwizzle128), idesc_qk,
+                               k > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&u_full[i & 1]);
+                }
+                if (i >= 1 && !pv_first && !issue_pv(i - 1)) break;
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax
+        const int sw = warp - 2;                 // 0 .. 4*NG-1
+        const int hg = sw >> 2;                  // head group (16 heads)
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;       // TMEM lane = tile row (key j, rank s)
+        const int jl = r / R, sr = r % R;
+        const int stid = threadIdx.x - 64;       // 0 .. NSM-1
+        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+        const int hbase = hg * 16;
+        float m[16], lp[16];
+        TileWalk<KT> tw;
+        if (n > 0) tw.init(P, g0);
+        int seg = -1, prev_b = -1;
+        // A failed (timed-out) wait only sets `bad`; the loop is left at the end of the
+        // tile by all softmax threads together (barrier 4), so that no thread is left
+        // waiting at a named barrier or a warp vote that the others have skipped.
+        bool bad = false;
+        for (int i = 0; i < n; ++i) {
+            const int g = g0 + i;
+            tw.advance(P, g);
+            const int b = tw.b;
+            const bool first = b != prev_b;
+            if (first) {
+                ++seg;
+                prev_b = b;
+                // q~ for this sequence into buffer seg&1 (K-major, 128-byte swizzle)
+                uint8_t* qb = qbuf + (size_t)(seg & 1) * kQW;
+                for (int e = stid; e < HH * (DH / 8); e += NSM) {
+                    const int h = e / (DH / 8), k8 = (e % (DH / 8)) * 8;
+                    float acc[8];
+                    if (a.Rq > 0) {
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+                        for (int rq = 0; rq < a.Rq; ++rq) {
+                            const float aqv = __bfloat162float(a.q_a[((long long)b * HH + h) * a.Rq + rq]);
+                            const uint4 raw = *reinterpret_cast<const uint4*>(a.q_b + ((long long)b * a.Rq + rq) * DH + k8);
+                            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                            for (int x = 0; x < 4; ++x) {
+                                const float2 f = __bfloat1622float2(p2[x]);
+                                acc[2 * x] = fmaf(aqv, f.x, acc[2 * x]);
+                                acc[2 * x + 1] = fmaf(aqv, f.y, acc[2 * x + 1]);
+                            }
+                        }
+                    } else {
+                        const uint4 raw = *reinterpret_cast<const uint4*>(a.q_b + ((long long)b * HH + h) * DH + k8);
+                        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            const float2 f = __bfloat1622float2(p2[x]);
+                            acc[2 * x] = f.x;
+                            acc[2 * x + 1] = f.y;
+                        }
+                    }
+                    uint4 w;
+                    w.x = pack_bf16(acc[0] * a.qscale, acc[1] * a.qscale);
+                    w.y = pack_bf16(acc[2] * a.qscale, acc[3] * a.qscale);
+                    w.z = pack_bf16(acc[4] * a.qscale, acc[5] * a.qscale);
+                    w.w = pack_bf16(acc[6] * a.qscale, acc[7] * a.qscale);
+                    *reinterpret_cast<uint4*>(qb + (k8 >> 6) * (HH * 128u) + sw128_offset(h, (k8 & 63) * 2)) = w;
+                }
+                fence_proxy_async_smem();
+                bar_sync(3, NSM);
+                if (stid == 0) mbar_arrive(&q_ready[seg & 1]);
+#pragma unroll
+                for (int h = 0; h < 16; ++h) { m[h] = -INFINITY; lp[h] = 0.f; }
+            }
+            const int j0 = (g - P.tile_prefix[b]) * KT;
+            const int len = P.len[b];
+            const bool valid = j0 + jl < len;
+            const int s = i % kStages;
+            if (!bad) bad = !mbar_wait(&u_full[i & 1], (uint32_t)((i >> 1) & 1), lim, a.err, abort);
+            if (!bad) bad = !mbar_wait(&kv_full[s], (uint32_t)((i / kStages) & 1), lim, a.err, abort);
+            tc_fence_after();
+            uint32_t u[16];
+            tmem_ld16(lane_addr + (uint32_t)(i & 1) * HH + hbase, u);
+            // this row's a^K and a^V for the group's 16 heads
+            float ak[16], av[16];
+            {
+                const __nv_bfloat16* akr = reinterpret_cast<const __nv_bfloat16*>(st_ak(s)) + ((size_t)jl * HH + hbase) * R;
+                const __nv_bfloat16* avr = reinterpret_cast<const __nv_bfloat16*>(st_av(s)) + ((size_t)jl * HH + hbase) * R;
+#pragma unroll
+                for (int h = 0; h < 16; ++h) {
+                    ak[h] = __bfloat162float(akr[h * R + sr]);
+                    av[h] = __bfloat162float(avr[h * R + sr]);
+                }
+            }
+            tmem_ld_wait();
+            float sc[16];
+            bool over = false;
+#pragma unroll
+            for (int h = 0; h < 16; ++h) {
+                float v = ak[h] * __uint_as_float(u[h]);
+#pragma unroll
+                for (int o = 1; o < R; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                sc[h] = valid ? v : -INFINITY;
+                over |= sc[h] - m[h] > kTau;
+            }
+            // first tile of a part, or a score above the reference max: exact tile max
+            if (bar_any(1 + hg, 128, first || over)) {
+                float* rd = red + hg * 64;
+#pragma unroll
+                for (int h = 0; h < 16; ++h) {
+                    float v = warp_max(sc[h]);
+                    if (lane == 0) rd[quarter * 16 + h] = v;
+                }
+                bar_sync(1 + hg, 128);
+                float alpha[16];
+                bool resc = false;
+#pragma unroll
+                for (int h = 0; h < 16; ++h) {
+                    const float mt = fmaxf(fmaxf(rd[h], rd[16 + h]), fmaxf(rd[32 + h], rd[48 + h]));
+                    const float mn = fmaxf(m[h], mt);
+                    alpha[h] = first ? 1.f : ex2(m[h] - mn);
+                    resc |= alpha[h] != 1.f;
+                    m[h] = mn;
+                    lp[h] *= alpha[h];
+                }
+                bar_sync(1 + hg, 128);                 // everyone has read the scratch
+                if (!first && __any_sync(0xffffffffu, resc)) {
+                    // O^T columns of this group *= alpha once PV(i-1) has completed
+                    if (!bad)
+                        bad = !mbar_wait(&w_empty[(i - 1) & 1], (uint32_t)(((i - 1) >> 1) & 1), lim, a.err, abort);
+                    tc_fence_after();
+                    uint32_t o[16];
+                    tmem_ld16(lane_addr + 2u * HH + hbase, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int h = 0; h < 16; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+                    tmem_st16(lane_addr + 2u * HH + hbase, o);
+                    tmem_st_wait();
+                }
+            }
+            // p and W^T (row r = K index, columns = heads), bf16 pairs of adjacent rows
+            if (i >= 2 && !bad)
+                bad = !mbar_wait(&w_empty[i & 1], (uint32_t)(((i >> 1) - 1) & 1), lim, a.err, abort);
+            uint8_t* wb = wbuf + (size_t)(i & 1) * kQW;
+#pragma unroll
+            for (int h = 0; h < 16; ++h) {
+                const float p = ex2(sc[h] - m[h]);
+                if (sr == 0) lp[h] += p;
+                const float w = valid ? p * av[h] : 0.f;
+                const float wn = __shfl_down_sync(0xffffffffu, w, 1);
+                if ((r & 1) == 0) {
+                    const int hh = hbase + h;
+                    *reinterpret_cast<uint32_t*>(wb + (r >> 6) * (HH * 128u) + sw128_offset(hh, (r & 63) * 2)) =
+                        pack_bf16(w, wn);
+                }
+            }
+            if (hg == 0 && !valid && j0 + jl >= len) {
+                // keys past the sequence: clear their b^V row so 0 * (cache contents) = 0
+                uint4* z0 = reinterpret_cast<uint4*>(st_bv(s) + r * 128);
+                uint4* z1 = reinterpret_cast<uint4*>(st_bv(s) + kBox + r * 128);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) { z0[e] = make_uint4(0, 0, 0, 0); z1[e] = make_uint4(0, 0, 0, 0); }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&w_full[i & 1]);
+            const bool last = (i == n - 1) || (P.tile_prefix[b + 1] <= g + 1);
+            if (last) {
+                // part done: O^T (lane = d row), l per head, written to the workspace
+                if (!bad) bad = !mbar_wait(o_done, (uint32_t)(seg & 1), lim, a.err, abort);
+                tc_fence_after();
+                uint32_t o[16];
+                tmem_ld16(lane_addr + 2u * HH + hbase, o);
+                tmem_ld_wait();
+                const int part = P.first_part[b] + (c - P.c_first[b]);
+                float* wo = a.ws_o + (size_t)part * HH * DH;
+                if (!bad) {
+#pragma unroll
+                    for (int h = 0; h < 16; ++h) wo[(size_t)(hbase + h) * DH + r] = __uint_as_float(o[h]);
+                }
+                float* rd = red + hg * 64;
+#pragma unroll
+                for (int h = 0; h < 16; ++h) {
+                    const float v = warp_sum(lp[h]);
+                    if (lane == 0) rd[quarter * 16 + h] = v;
+                }
+                bar_sync(1 + hg, 128);
+                if (r < 16 && !bad) {
+                    const float l = (rd[r] + rd[16 + r]) + (rd[32 + r] + rd[48 + r]);
+                    a.ws_ml[((size_t)part * HH + hbase + r) * 2 + 0] = m[r];
+                    a.ws_ml[((size_t)part * HH + hbase + r) * 2 + 1] = l;
+                }
+                bar_sync(1 + hg, 128);
+                tc_fence_before();
+                mbar_arrive(o_free);
+            }
+            if (bar_any(4, NSM, bad)) break;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
 }
+
+template <int HH, int R>
+cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const DecodePlan& plan,
+                     cudaStream_t st) {
+    constexpr int KT = 128 / R;
+    a.a_bytes = (uint32_t)(KT * HH * R * 2);
+    const uint32_t a_pad = (a.a_bytes + 127u) & ~127u;
+    a.stage_bytes = ((4u * kBox + 2u * a_pad) + 1023u) & ~1023u;
+    const size_t smem = 1024 + (size_t)kStages * a.stage_bytes + 4u * HH * 256u +
+                        (HH / 16) * 64 * sizeof(float) + 32 * 8 + 16;
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
+    CUtensorMap tmk, tmv;
+    const uint64_t dims[2] = {(uint64_t)DH, (uint64_t)c.batch * c.capacity * R};
+    const uint64_t stride[1] = {(uint64_t)DH * 2};
+    const uint32_t box[2] = {64, 128};
+    if (!make_tmap_bf16(&tmk, c.b_k, 2, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 2, dims, stride, box))
+        return cudaErrorInvalidValue;
+    constexpr int threads = 64 + 32 * 4 * (HH / 16);
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<HH, R>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    decode_tc_kernel<HH, R><<<plan.n_ctas, threads, smem, st>>>(tmk, tmv, a, plan);
+    return cudaGetLastError();
+}
+}  // namespace
+
+bool decode_tc_supported(const Shape& s) {
+    return s.bf16 && s.Dh == DH && (s.H == 16 || s.H == 32) && s.Rk == 2 && s.Rv == 2 &&
+           s.Rq <= 64;
+}
+
+cudaError_t launch_decode_tc(const Shape& s, const void* q_a, const void* q_b, const tpa_cache& c,
+                             const DecodePlan& plan, float* ws, int* err, uint32_t wait_limit,
+                             cudaStream_t st) {
+    if ((long long)c.batch * c.capacity * s.Rk >= (1LL << 31)) return cudaErrorInvalidValue;
+    if (plan.total_tiles < 1 || plan.n_ctas < 1) return cudaErrorInvalidValue;
+    DecodeTcArgs a{};
+    a.q_a = static_cast<const __nv_bfloat16*>(q_a);
+    a.q_b = static_cast<const __nv_bfloat16*>(q_b);
+    a.ca_k = static_cast<const __nv_bfloat16*>(c.a_k);
+    a.ca_v = static_cast<const __nv_bfloat16*>(c.a_v);
+    a.ws_ml = ws;
+    a.ws_o = ws + (size_t)plan.total_parts * s.H * 2;
+    a.Rq = s.Rq;
+    a.cap = c.capacity;
+    a.qscale = 1.4426950408889634f / ((s.Rq > 0 ? (float)s.Rq : 1.f) * (float)s.Rk * std::sqrt((float)s.Dh));
+    a.err = err;
+    a.wait_limit = wait_limit;
+    if (s.H == 16) return launch_t<16, 2>(s, a, c, plan, st);
+    return launch_t<32, 2>(s, a, c, plan, st);
+}
+
 }  // namespace tpa

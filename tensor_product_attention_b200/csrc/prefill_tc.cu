@@ -351,7 +351,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         bool alive = true;
         const uint32_t u_addr = lane_addr + u_col;
         for (int t = 0; t < n_tiles; ++t) {
-            if (!mbar_wait(&u_ready[bl], (uint32_t)(t & 1), lim, a.err, abort)) { alive = false; break; }
+            // leave together: the warp votes below need every lane
+            const bool got = mbar_wait(&u_ready[bl], (uint32_t)(t & 1), lim, a.err, abort);
+            if (__any_sync(0xffffffffu, !got)) { alive = false; break; }
             tc_fence_after();
             const int s = t % a.stages;
             const int j0 = t * KT;
@@ -416,7 +418,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             tc_fence_before();
             mbar_arrive(&w_ready[bl]);
         }
-        if (alive && mbar_wait(&o_done[bl], 0u, lim, a.err, abort)) {
+        const bool fin = alive && mbar_wait(&o_done[bl], 0u, lim, a.err, abort);
+        if (__all_sync(0xffffffffu, fin)) {
             tc_fence_after();
             const float inv = a.out_scale / l;
             const long long t = (long long)b * a.S + q0 + i_loc;

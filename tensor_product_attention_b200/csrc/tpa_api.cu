@@ -190,7 +190,9 @@ size_t tpa_decode_workspace_bytes(const tpa_dims* d, const int32_t* lengths, int
     for (int b = 0; b < batch; ++b)
         if (lengths[b] < 1) return 0;
     Shape s = shape_of(*d);
-    return decode_workspace_bytes(s, decode_schedule(s, lengths, batch), batch);
+    DecodePlan plan;
+    make_decode_plan(s, lengths, batch, s.bf16 && decode_tc_supported(s), &plan);
+    return decode_workspace_bytes(s, plan);
 }
 
 tpa_status tpa_decode(const tpa_dims* d, const void* q_a, const void* q_b,
@@ -203,27 +205,23 @@ tpa_status tpa_decode(const tpa_dims* d, const void* q_a, const void* q_b,
     if (d->rank_q > 0 && (!q_a || !aligned16(q_a))) return TPA_ERR_INVALID;
     if (!aligned16(q_b) || !aligned16(out) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return TPA_ERR_INVALID;
-    SeqParams sp;
     for (int b = 0; b < batch; ++b) {
         if (lengths[b] < 1) return TPA_ERR_INVALID;
         if (lengths[b] > c->capacity) return TPA_ERR_CAPACITY;
-        sp.v[b] = lengths[b];
     }
     Shape s = shape_of(*d);
-    DecodeSchedule sch = decode_schedule(s, lengths, batch);
-    if (decode_workspace_bytes(s, sch, batch) > workspace_bytes) return TPA_ERR_WORKSPACE;
+    const bool tc = s.bf16 && decode_tc_supported(s);
+    if (!tc && (long long)s.H * s.Dh > 8192) return TPA_ERR_UNSUPPORTED;
+    DecodePlan plan;
+    make_decode_plan(s, lengths, batch, tc, &plan);
+    if (decode_workspace_bytes(s, plan) > workspace_bytes) return TPA_ERR_WORKSPACE;
     cudaStream_t cs = (cudaStream_t)stream;
     float* ws = static_cast<float*>(workspace);
-    cudaError_t e;
-    if (s.bf16 && decode_tc_supported(s)) {
-        e = launch_decode_tc(s, q_a, q_b, *c, sp, batch, sch, ws, device_error_ptr(),
-                             wait_limit(), cs);
-    } else {
-        if ((long long)s.H * s.Dh > 8192) return TPA_ERR_UNSUPPORTED;
-        e = launch_decode_simt(s, q_a, q_b, *c, sp, batch, sch, ws, cs);
-    }
+    cudaError_t e = tc ? launch_decode_tc(s, q_a, q_b, *c, plan, ws, device_error_ptr(),
+                                          wait_limit(), cs)
+                       : launch_decode_simt(s, q_a, q_b, *c, plan, ws, cs);
     if (e != cudaSuccess) return TPA_ERR_CUDA;
-    return launched(launch_decode_combine(s, sp, batch, sch, ws, out, cs));
+    return launched(launch_decode_combine(s, plan, ws, out, cs));
 }
 
 tpa_status tpa_get_device_error(tpa_stream_t stream, int32_t* code) {

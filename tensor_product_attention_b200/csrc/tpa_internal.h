@@ -41,14 +41,27 @@ inline ProjLayout proj_layout(const Shape& s, const tpa_factors& f) {
     return L;
 }
 
-// Decode split schedule: sequence b is cut into ceil(len_b / split_len) pieces.
-struct DecodeSchedule {
-    int split_len;      // keys per split (multiple of the kernel's key tile)
-    int max_splits;     // grid.x
+// Decode plan.  Each sequence's context is cut into pieces ("parts"); every part
+// leaves one partial softmax state (m, l, o) per head in the workspace, and the
+// combine kernel merges the parts of a sequence in part order.  The parts of
+// sequence b are first_part[b] .. first_part[b] + n_parts[b] - 1.
+//  - CUDA-core decode: parts are splits of split_len keys; CTA (split, b).
+//  - tensor-core decode: a persistent grid of n_ctas CTAs walks the concatenated
+//    key tiles of all sequences; CTA c takes tiles [c*N/G, (c+1)*N/G), and each
+//    (CTA, sequence) overlap is one part; c_first[b] is the first CTA on sequence b.
+struct DecodePlan {
+    int32_t len[TPA_MAX_BATCH];
+    int32_t first_part[TPA_MAX_BATCH];
+    int32_t n_parts[TPA_MAX_BATCH];
+    int32_t tile_prefix[TPA_MAX_BATCH + 1];
+    int32_t c_first[TPA_MAX_BATCH];
+    int32_t batch, n_ctas, total_tiles, total_parts, split_len, key_tile;
 };
 
-DecodeSchedule decode_schedule(const Shape& s, const int32_t* lengths, int batch);
-size_t decode_workspace_bytes(const Shape& s, const DecodeSchedule& sch, int batch);
+// Builds the plan for the decode kernel that handles this shape (tc = tensor-core path).
+void make_decode_plan(const Shape& s, const int32_t* lengths, int batch, bool tc,
+                      DecodePlan* plan);
+size_t decode_workspace_bytes(const Shape& s, const DecodePlan& plan);
 
 // ---- launchers (each returns the launch's cudaError_t) ----
 cudaError_t launch_rope_table(float* cs, int max_pos, int head_dim, double base,
@@ -78,17 +91,15 @@ cudaError_t launch_prefill_tc(const Shape& s, const tpa_factors& q, const tpa_ca
 bool prefill_tc_supported(const Shape& s);
 
 cudaError_t launch_decode_simt(const Shape& s, const void* q_a, const void* q_b,
-                               const tpa_cache& c, const SeqParams& len, int batch,
-                               const DecodeSchedule& sch, float* ws, cudaStream_t st);
+                               const tpa_cache& c, const DecodePlan& plan, float* ws,
+                               cudaStream_t st);
 
 cudaError_t launch_decode_tc(const Shape& s, const void* q_a, const void* q_b,
-                             const tpa_cache& c, const SeqParams& len, int batch,
-                             const DecodeSchedule& sch, float* ws, int* err,
+                             const tpa_cache& c, const DecodePlan& plan, float* ws, int* err,
                              uint32_t wait_limit, cudaStream_t st);
 bool decode_tc_supported(const Shape& s);
 
-cudaError_t launch_decode_combine(const Shape& s, const SeqParams& len, int batch,
-                                  const DecodeSchedule& sch, const float* ws, void* out,
-                                  cudaStream_t st);
+cudaError_t launch_decode_combine(const Shape& s, const DecodePlan& plan, const float* ws,
+                                  void* out, cudaStream_t st);
 
 }  // namespace tpa

@@ -93,6 +93,8 @@ def test_workspace_size_formula(bnd):
     dims = bnd.Dims(0, 16, 128, 6, 2, 2)
     lengths = [32768] * 64
     n = bnd.tpa_decode_workspace_bytes(dims, lengths)
-    # one (m, l) pair and one d_h-vector of fp32 per (sequence, split, head)
-    per_split = 16 * (128 + 2) * 4
-    assert n % (64 * per_split) == 0 and n > 0
+    # one (m, l) pair and one d_h-vector of fp32 per (part, head); every sequence has at
+    # least one part, and a persistent grid of G CTAs adds at most G more
+    per_part = 16 * (128 + 2) * 4
+    assert n % per_part == 0
+    assert 64 * per_part <= n <= (64 + 1024) * per_part
