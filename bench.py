@@ -321,13 +321,22 @@ class DecodeStep:
 
 # ------------------------------------------------------------------ timing
 
-def timed(step, steps, warmup, ws, flush: torch.Tensor | None):
-    """W untimed steps, then exactly K timed steps between barrier+sync; per-step CUDA
-    events on the launching stream (the L2 flush, when used, sits between steps and
-    outside the events).  Returns (per-step ms averaged over K, max over ranks; events)."""
+def timed(step, steps, warmup, ws, flush: torch.Tensor | None, graph: bool = True):
+    """W untimed steps, then exactly K timed steps between barrier+sync, each timed
+    with CUDA events on the launching stream.  With `graph`, the step's launches are
+    captured once into a CUDA graph and the K timed steps are graph replays (the
+    host-side argument checks and launch overhead stay out of the step).  The L2
+    flush, when used, sits between steps and outside the events.  Returns the mean
+    per-step ms (max over ranks)."""
     for _ in range(warmup):
         step.run()
     torch.cuda.synchronize()
+    g = None
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step.run()
+        torch.cuda.synchronize()
     ev = Events()
     barrier(ws)
     torch.cuda.synchronize()
@@ -335,12 +344,27 @@ def timed(step, steps, warmup, ws, flush: torch.Tensor | None):
         if flush is not None:
             flush.zero_()
         ev.start("step")
-        step.run(ev)
+        if g is not None:
+            g.replay()
+        else:
+            step.run()
         ev.stop("step")
     torch.cuda.synchronize()
     barrier(ws)
     ms = ev.total_ms("step") / steps
-    return max_over_ranks(ws, ms), ev
+    del g
+    return max_over_ranks(ws, ms)
+
+
+def timed_legs(step, steps, flush: torch.Tensor | None):
+    """Per-call CUDA events for each leg of the step (direct calls, not a graph)."""
+    ev = Events()
+    for _ in range(steps):
+        if flush is not None:
+            flush.zero_()
+        step.run(ev)
+    torch.cuda.synchronize()
+    return ev
 
 
 def timed_e2e(step, steps, warmup, ws):
@@ -451,6 +475,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode-leg", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time direct calls instead of graph replays")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -469,7 +494,8 @@ def main():
     step = PrefillStep(wl, tpa) if wl.kind == "prefill" else DecodeStep(wl, tpa)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if wl.kind == "prefill" else None
     with ClockSampler(local) as clk:
-        ms, ev = timed(step, args.steps, args.warmup, ws, flush)
+        ms = timed(step, args.steps, args.warmup, ws, flush, graph=not args.no_graph)
+        ev = timed_legs(step, args.steps, flush)
         e2e_ms = timed_e2e(step, args.steps, args.warmup, ws)
     clocks = clk.summary()
     assert tpa.tpa_get_device_error() == 0
@@ -495,6 +521,7 @@ def main():
                   "rank_k": wl.rank_k, "rank_v": wl.rank_v,
                   "step": "project+RoPE -> append -> causal prefill, then 1 decode token per sequence",
                   "l2": "flushed between steps (256 MiB write outside the step events)",
+                  "timing": "CUDA-graph replay of the step" if not args.no_graph else "direct calls",
                   "parallelism": f"dp{ws} (independent sequences per rank)"}
     else:
         work = step.bytes()
@@ -511,6 +538,7 @@ def main():
         config = {"workload": wl.name, "batch": wl.batch, "context": list(wl.context),
                   "n_heads": wl.n_heads, "head_dim": wl.head_dim, "rank_q": wl.rank_q,
                   "rank_k": wl.rank_k, "rank_v": wl.rank_v, "l2": "inputs larger than L2",
+                  "timing": "CUDA-graph replay of the step" if not args.no_graph else "direct calls",
                   "parallelism": f"dp{ws} (independent sequences per rank)"}
     h2d, d2h = step.io_bytes()
     line = {
@@ -528,7 +556,8 @@ def main():
     if wl.kind == "prefill" and not args.no_decode_leg:
         dl = I.WORKLOADS[DECODE_LEG]
         dstep = DecodeStep(dl, tpa)
-        dms, dev = timed(dstep, args.steps, args.warmup, ws, None)
+        dms = timed(dstep, args.steps, args.warmup, ws, None, graph=not args.no_graph)
+        dev = timed_legs(dstep, args.steps, None)
         dval = ws * dstep.bytes() / (dms * 1e-3) / 1e9
         dach = dstep.factor_bytes() / (dev.mean_ms("decode") * 1e-3) / 1e9
         line["decode_leg"] = {"workload": dl.name, "value": dval, "unit": "GB/s", "ms_per_step": dms,

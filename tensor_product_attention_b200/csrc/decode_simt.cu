@@ -285,13 +285,11 @@ cudaError_t launch_decode_simt(const Shape& s, const void* q_a, const void* q_b,
     dim3 grid(plan.n_ctas, plan.batch);
     cudaError_t e;
     if (s.bf16) {
-        e = cudaFuncSetAttribute(decode_simt_kernel<__nv_bfloat16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = allow_smem(reinterpret_cast<const void*>(decode_simt_kernel<__nv_bfloat16>), (int)smem);
         if (e != cudaSuccess) return e;
         decode_simt_kernel<__nv_bfloat16><<<grid, NT, smem, st>>>(a, plan);
     } else {
-        e = cudaFuncSetAttribute(decode_simt_kernel<float>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = allow_smem(reinterpret_cast<const void*>(decode_simt_kernel<float>), (int)smem);
         if (e != cudaSuccess) return e;
         decode_simt_kernel<float><<<grid, NT, smem, st>>>(a, plan);
     }

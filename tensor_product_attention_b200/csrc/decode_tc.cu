@@ -35,7 +35,6 @@ namespace tpa {
 namespace {
 using namespace sm100;
 
-constexpr int DH = 128;                  // head dim (M of the value MMA)
 constexpr uint32_t kBox = 128 * 128;     // one TMA box: 128 rows x 128 bytes
 constexpr float kTau = 8.f;              // lazy rescale threshold (log2 units)
 constexpr int kStages = 2;
@@ -67,11 +66,12 @@ struct TileWalk {
     }
 };
 
-template <int HH, int R>
+template <int DH, int HH, int R>
 __global__ void __launch_bounds__(64 + 32 * 4 * (HH / 16), 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                  const DecodeTcArgs a, const DecodePlan P) {
     constexpr int KT = 128 / R;                 // keys per tile
+    constexpr int NB = DH / 64;                 // 64-wide column blocks of d_h (1 or 2)
     constexpr int NG = HH / 16;                 // head groups of 16 (4 warps each)
     constexpr int NSM = 128 * NG;               // softmax threads
     constexpr uint32_t kQW = HH * 256u;         // q~ or W^T buffer: 2 x [HH rows][128 B]
@@ -146,12 +146,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     break;
                 const int rows_a = min(KT, a.cap - j0);
                 const uint32_t abytes = (uint32_t)rows_a * HH * R * 2u;
-                mbar_arrive_expect_tx(&kv_full[s], 4u * kBox + 2u * abytes);
+                mbar_arrive_expect_tx(&kv_full[s], (NB + 2u) * kBox + 2u * abytes);
                 const int y = (int)(((long long)b * a.cap + j0) * R);
                 tma_load_2d(st_bk(s), &tmk, &kv_full[s], 0, y);
-                tma_load_2d(st_bk(s) + kBox, &tmk, &kv_full[s], 64, y);
+                if (NB == 2) tma_load_2d(st_bk(s) + kBox, &tmk, &kv_full[s], 64, y);
+                // the value MMA has M = 128 rows of d_h: for d_h = 64 the one box is
+                // loaded twice and output rows 64..127 (a copy of 0..63) are dropped
                 tma_load_2d(st_bv(s), &tmv, &kv_full[s], 0, y);
-                tma_load_2d(st_bv(s) + kBox, &tmv, &kv_full[s], 64, y);
+                tma_load_2d(st_bv(s) + kBox, &tmv, &kv_full[s], NB == 2 ? 64 : 0, y);
                 const long long ea = ((long long)b * a.cap + j0) * HH * R;
                 bulk_load(st_ak(s), a.ca_k + ea, abytes, &kv_full[s]);
                 bulk_load(st_av(s), a.ca_v + ea, abytes, &kv_full[s]);
@@ -405,7 +407,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 tmem_ld_wait();
                 const int part = P.first_part[b] + (c - P.c_first[b]);
                 float* wo = a.ws_o + (size_t)part * HH * DH;
-                if (!bad) {
+                if (!bad && r < DH) {
 #pragma unroll
                     for (int h = 0; h < 16; ++h) wo[(size_t)(hbase + h) * DH + r] = __uint_as_float(o[h]);
                 }
@@ -436,7 +438,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     }
 }
 
-template <int HH, int R>
+template <int DH, int HH, int R>
 cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const DecodePlan& plan,
                      cudaStream_t st) {
     constexpr int KT = 128 / R;
@@ -453,17 +455,16 @@ cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const D
     if (!make_tmap_bf16(&tmk, c.b_k, 2, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 2, dims, stride, box))
         return cudaErrorInvalidValue;
     constexpr int threads = 64 + 32 * 4 * (HH / 16);
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<HH, R>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = allow_smem(reinterpret_cast<const void*>(decode_tc_kernel<DH, HH, R>), (int)smem);
     if (e != cudaSuccess) return e;
-    decode_tc_kernel<HH, R><<<plan.n_ctas, threads, smem, st>>>(tmk, tmv, a, plan);
+    decode_tc_kernel<DH, HH, R><<<plan.n_ctas, threads, smem, st>>>(tmk, tmv, a, plan);
     return cudaGetLastError();
 }
 }  // namespace
 
 bool decode_tc_supported(const Shape& s) {
-    return s.bf16 && s.Dh == DH && (s.H == 16 || s.H == 32) && s.Rk == 2 && s.Rv == 2 &&
-           s.Rq <= 64;
+    return s.bf16 && (s.Dh == 64 || s.Dh == 128) && (s.H == 16 || s.H == 32) && s.Rk == 2 &&
+           s.Rv == 2 && s.Rq <= 64;
 }
 
 cudaError_t launch_decode_tc(const Shape& s, const void* q_a, const void* q_b, const tpa_cache& c,
@@ -483,8 +484,9 @@ cudaError_t launch_decode_tc(const Shape& s, const void* q_a, const void* q_b, c
     a.qscale = 1.4426950408889634f / ((s.Rq > 0 ? (float)s.Rq : 1.f) * (float)s.Rk * std::sqrt((float)s.Dh));
     a.err = err;
     a.wait_limit = wait_limit;
-    if (s.H == 16) return launch_t<16, 2>(s, a, c, plan, st);
-    return launch_t<32, 2>(s, a, c, plan, st);
+    if (s.Dh == 64) return s.H == 16 ? launch_t<64, 16, 2>(s, a, c, plan, st)
+                                     : launch_t<64, 32, 2>(s, a, c, plan, st);
+    return s.H == 16 ? launch_t<128, 16, 2>(s, a, c, plan, st) : launch_t<128, 32, 2>(s, a, c, plan, st);
 }
 
 }  // namespace tpa

@@ -471,8 +471,7 @@ cudaError_t launch_t(const PrefillTcArgs& a0, const tpa_cache& c, int batch, con
     if (!make_tmap_bf16(&tmk, c.b_k, 2, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 2, dims, stride, box))
         return cudaErrorInvalidValue;
     const size_t smem = 1024 + q_bytes + (size_t)a.stages * a.stage_bytes + (2 * a.stages + 6) * 8 + 16;
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<DH, R, HC>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = allow_smem(reinterpret_cast<const void*>(prefill_tc_kernel<DH, R, HC>), (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.n_qblocks, batch);
     prefill_tc_kernel<DH, R, HC><<<grid, kThreads, smem, st>>>(tmk, tmv, a, start);

@@ -276,8 +276,7 @@ cudaError_t launch_project_tc(const Shape& s, const void* x, const void* w, int 
         return cudaErrorInvalidValue;
 
     const size_t smem = 1024 + (size_t)a.stages * stage_bytes + (2 * a.stages + 4) * 8 + 16;
-    cudaError_t e = cudaFuncSetAttribute(project_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = allow_smem(reinterpret_cast<const void*>(project_tc_kernel), (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = std::min(a.n_tiles, sm_count());
     project_tc_kernel<<<grid, kThreads, smem, st>>>(tmx, tmw, a, start);

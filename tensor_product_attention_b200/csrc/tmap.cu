@@ -39,11 +39,32 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t
     return r == CUDA_SUCCESS;
 }
 
+cudaError_t allow_smem(const void* func, int bytes) {
+    struct Entry { const void* f; int dev; int bytes; };
+    static Entry table[64];
+    static int used = 0;
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+        if (table[i].f == func && table[i].dev == dev && table[i].bytes >= bytes) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    for (int i = 0; i < used; ++i)
+        if (table[i].f == func && table[i].dev == dev) { table[i].bytes = bytes; return e; }
+    if (used < 64) table[used++] = Entry{func, dev, bytes};
+    return e;
+}
+
 int sm_count() {
+    static int cached[64] = {};
     int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return n;
+    if (cached[dev] > 0) return cached[dev];
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+    return n;
 }
 
 }  // namespace tpa

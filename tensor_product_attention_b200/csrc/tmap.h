@@ -15,4 +15,8 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t
 
 int sm_count();
 
+// Raise `func`'s dynamic shared-memory limit to at least `bytes` on the current
+// device.  Remembered per (kernel, device), so repeated launches skip the call.
+cudaError_t allow_smem(const void* func, int bytes);
+
 }  // namespace tpa

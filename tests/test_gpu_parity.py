@@ -162,6 +162,9 @@ DECODE_CASES = [
     (I.custom("d_multi", C3), [12000, 9001, 1, 14500], 1.0),
     (I.custom("d_multi", C3), [700] * 29 + [33], 8.0),
     (I.custom("d_kvmulti", C4), [20000, 13001], 8.0),
+    # head_dim 64 (the value MMA repeats the 64-wide tile to fill its 128 rows)
+    (I.custom("d_d64", C3, head_dim=64), [2049, 1, 700], 8.0),
+    (I.custom("d_d64", C3, head_dim=64), [9000] * 8, 1.0),
 ]
 
 
