@@ -41,6 +41,15 @@ DEFAULT = "prefill_b8_s2048_d1024"
 DECODE_LEG = "decode_b64_ctx32k"
 FLUSH_BYTES = 256 << 20          # > 126 MB L2
 
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture of
+# the kernel as it stands (dram__bytes_read.sum + dram__bytes_write.sum); None where no
+# capture of the current kernel exists.  The 32K decode was captured on 16 of its 64
+# sequences and scaled by the keys processed (traffic grows in proportion).
+PROFILED_TRAFFIC = {
+    ("prefill_b8_s2048_d1024", "tpa_prefill"): 26.53e6,
+    ("decode_b64_ctx32k", "tpa_decode"): 4 * 609.42e6,
+}
+
 
 # ------------------------------------------------------------------ accounting
 
@@ -510,7 +519,7 @@ def main():
         ach = pre_fl / (pre_ms * 1e-3) / 1e12
         roof = {"kernel": "tpa_prefill (causal attention from factors)", "bound": "tensor",
                 "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach / pk["bf16_tflops"], "traffic": None,
+                "frac": ach / pk["bf16_tflops"], "traffic": PROFILED_TRAFFIC.get((wl.name, "tpa_prefill")),
                 "peak_kind": f"bf16 dense, burst, {pk['source']}",
                 "algorithmic_per_launch": f"{pre_fl:.4g} flop = {attn_flops_per_pair(wl)} flop/pair x "
                                           f"{causal_pairs(wl.batch, wl.seqlen)} causal pairs",
@@ -530,7 +539,8 @@ def main():
         unit = "GB/s"
         ach = step.factor_bytes() / (ev.mean_ms("decode") * 1e-3) / 1e9
         roof = {"kernel": "tpa_decode (split-K decode + combine)", "bound": "hbm", "achieved": ach,
-                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"], "traffic": None,
+                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
+                "traffic": PROFILED_TRAFFIC.get((wl.name, "tpa_decode")),
                 "peak_kind": f"HBM copy, {pk['source']}",
                 "algorithmic_per_launch": f"{step.factor_bytes()} factor bytes",
                 "launch_ms": ev.mean_ms("decode")}
@@ -562,6 +572,7 @@ def main():
         dach = dstep.factor_bytes() / (dev.mean_ms("decode") * 1e-3) / 1e9
         line["decode_leg"] = {"workload": dl.name, "value": dval, "unit": "GB/s", "ms_per_step": dms,
                               "frac_of_hbm": dach / pk["hbm_gbs"], "factor_bytes": dstep.factor_bytes(),
+                              "traffic": PROFILED_TRAFFIC.get((dl.name, "tpa_decode")),
                               "gpu_launches": dstep.launches_per_step * args.steps}
         line["gpu_launches"] += dstep.launches_per_step * args.steps
         del dstep
