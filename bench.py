@@ -171,12 +171,20 @@ def barrier(ws):
 
 
 def max_over_ranks(ws, value: float) -> float:
+    """The slowest rank's time: every rank gets the max (timing plumbing only)."""
     if ws == 1:
         return value
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(ws: int, work_per_rank: float, ms_max: float) -> float:
+    """Weak scaling: every rank processes its own batch of `work_per_rank` units; the
+    job rate is all ranks' units over the slowest rank's time (per second)."""
+    return ws * work_per_rank / (ms_max * 1e-3)
 
 
 class Events:
@@ -511,8 +519,8 @@ def main():
 
     if wl.kind == "prefill":
         work = step.flops()
-        value = ws * work / (ms * 1e-3) / 1e12
-        e2e_v = ws * work / (e2e_ms * 1e-3) / 1e12
+        value = whole_job_rate(ws, work, ms) / 1e12
+        e2e_v = whole_job_rate(ws, work, e2e_ms) / 1e12
         unit = "TFLOP/s"
         pre_ms = ev.mean_ms("prefill")
         pre_fl = attn_flops_per_pair(wl) * causal_pairs(wl.batch, wl.seqlen)
@@ -534,8 +542,8 @@ def main():
                   "parallelism": f"dp{ws} (independent sequences per rank)"}
     else:
         work = step.bytes()
-        value = ws * work / (ms * 1e-3) / 1e9
-        e2e_v = ws * work / (e2e_ms * 1e-3) / 1e9
+        value = whole_job_rate(ws, work, ms) / 1e9
+        e2e_v = whole_job_rate(ws, work, e2e_ms) / 1e9
         unit = "GB/s"
         ach = step.factor_bytes() / (ev.mean_ms("decode") * 1e-3) / 1e9
         roof = {"kernel": "tpa_decode (split-K decode + combine)", "bound": "hbm", "achieved": ach,
@@ -568,7 +576,7 @@ def main():
         dstep = DecodeStep(dl, tpa)
         dms = timed(dstep, args.steps, args.warmup, ws, None, graph=not args.no_graph)
         dev = timed_legs(dstep, args.steps, None)
-        dval = ws * dstep.bytes() / (dms * 1e-3) / 1e9
+        dval = whole_job_rate(ws, dstep.bytes(), dms) / 1e9
         dach = dstep.factor_bytes() / (dev.mean_ms("decode") * 1e-3) / 1e9
         line["decode_leg"] = {"workload": dl.name, "value": dval, "unit": "GB/s", "ms_per_step": dms,
                               "frac_of_hbm": dach / pk["hbm_gbs"], "factor_bytes": dstep.factor_bytes(),

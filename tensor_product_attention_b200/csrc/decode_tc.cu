@@ -92,7 +92,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     uint64_t* q_ready = w_empty + 2;             // [2]
     uint64_t* o_done = q_ready + 2;              // [1]
     uint64_t* o_free = o_done + 1;               // [1]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 1);
+    uint64_t* fin = o_free + 1;                  // MMAs in flight at exit
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     auto st_bk = [&](int s) { return stg + (size_t)s * a.stage_bytes; };
@@ -119,6 +120,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         }
         mbar_init(o_done, 1);
         mbar_init(o_free, NSM);
+        mbar_init(fin, 1);
         *abort = 0;
         fence_mbar_init();
     }
@@ -161,8 +163,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             for (int s = 0; s < kStages; ++s) {                 // drain issued copies
                 const int fills = i > s ? (i - s - 1) / kStages + 1 : 0;
                 if (fills > 0)
-                    for (uint32_t k = 0; k < lim; ++k)
-                        if (mbar_try_wait(&kv_full[s], (uint32_t)((fills - 1) & 1))) break;
+                    drain_wait(&kv_full[s], (uint32_t)((fills - 1) & 1));
             }
         }
     } else if (warp == 1) {
@@ -236,6 +237,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 }
                 if (i >= 1 && !pv_first && !issue_pv(i - 1)) break;
             }
+            // every MMA issued has completed before TMEM is released
+            mma_commit(fin);
+            drain_wait(fin, 0);
         }
     } else {
         // ---------------------------------------------------------------- softmax

@@ -175,7 +175,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     uint64_t* u_ready = kv_empty + a.stages;    // [2]
     uint64_t* w_ready = u_ready + 2;            // [2]
     uint64_t* o_done = w_ready + 2;             // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 2);
+    uint64_t* fin = o_done + 2;                 // MMAs in flight at exit
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -207,6 +208,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             mbar_init(&w_ready[i], 128);
             mbar_init(&o_done[i], 1);
         }
+        mbar_init(fin, 1);
         *abort = 0;
         fence_mbar_init();
     }
@@ -278,8 +280,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             for (int s = 0; s < a.stages; ++s) {          // drain issued copies
                 const int fills = t > s ? (t - s - 1) / a.stages + 1 : 0;
                 if (fills > 0)
-                    for (uint32_t i = 0; i < lim; ++i)
-                        if (mbar_try_wait(&kv_full[s], (uint32_t)((fills - 1) & 1))) break;
+                    drain_wait(&kv_full[s], (uint32_t)((fills - 1) & 1));
             }
         }
       } else if (warp == 1) {
@@ -332,6 +333,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 }
                 if (!ok) break;
             }
+            // every MMA issued has completed before TMEM is released
+            mma_commit(fin);
+            drain_wait(fin, 0);
         }
       }
     } else {
@@ -470,7 +474,7 @@ cudaError_t launch_t(const PrefillTcArgs& a0, const tpa_cache& c, int batch, con
     const uint32_t box[2] = {64, 128};
     if (!make_tmap_bf16(&tmk, c.b_k, 2, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 2, dims, stride, box))
         return cudaErrorInvalidValue;
-    const size_t smem = 1024 + q_bytes + (size_t)a.stages * a.stage_bytes + (2 * a.stages + 6) * 8 + 16;
+    const size_t smem = 1024 + q_bytes + (size_t)a.stages * a.stage_bytes + (2 * a.stages + 7) * 8 + 16;
     cudaError_t e = allow_smem(reinterpret_cast<const void*>(prefill_tc_kernel<DH, R, HC>), (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.n_qblocks, batch);

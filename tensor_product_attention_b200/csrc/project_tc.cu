@@ -89,13 +89,15 @@ project_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
     uint64_t* empty = full + a.stages;
     uint64_t* tfull = empty + a.stages;     // [2] accumulator ready
     uint64_t* tempty = tfull + 2;           // [2] accumulator drained
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    uint64_t* fin = tempty + 2;             // MMAs in flight at exit
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < a.stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 8); }
+        mbar_init(fin, 1);
         *abort = 0;
         fence_mbar_init();
     }
@@ -126,8 +128,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
             for (int s = 0; s < a.stages; ++s) {
                 const long long fills = it > s ? (it - s - 1) / a.stages + 1 : 0;
                 if (fills > 0) {
-                    for (uint32_t i = 0; i < lim; ++i)
-                        if (mbar_try_wait(&full[s], (uint32_t)((fills - 1) & 1))) break;
+                    drain_wait(&full[s], (uint32_t)((fills - 1) & 1));
                 }
             }
         }
@@ -164,6 +165,9 @@ project_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
                 if (!ok) break;
                 mma_commit(&tfull[buf]);
             }
+            // every MMA issued has completed before TMEM is released
+            mma_commit(fin);
+            drain_wait(fin, 0);
         }
     } else {
         // 8 epilogue warps: warp w reads TMEM lanes 32*(w%4).. (its rows) and every
@@ -175,7 +179,9 @@ project_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
         int local = 0;
         for (int tile = blockIdx.x; tile < a.n_tiles; tile += gridDim.x, ++local) {
             const int buf = local & 1;
-            if (!mbar_wait(&tfull[buf], (uint32_t)((local >> 1) & 1), lim, a.err, abort)) break;
+            // leave together: tcgen05.ld below needs every lane
+            const bool got = mbar_wait(&tfull[buf], (uint32_t)((local >> 1) & 1), lim, a.err, abort);
+            if (__any_sync(0xffffffffu, !got)) break;
             tc_fence_after();
             const int m = tile / a.n_tiles_n, n = tile - m * a.n_tiles_n;
             const long long t = (long long)m * BM + row;
@@ -275,7 +281,7 @@ cudaError_t launch_project_tc(const Shape& s, const void* x, const void* w, int 
     if (!make_tmap_bf16(&tmx, x, 2, dx, stride, bx) || !make_tmap_bf16(&tmw, w, 2, dw, stride, bw))
         return cudaErrorInvalidValue;
 
-    const size_t smem = 1024 + (size_t)a.stages * stage_bytes + (2 * a.stages + 4) * 8 + 16;
+    const size_t smem = 1024 + (size_t)a.stages * stage_bytes + (2 * a.stages + 5) * 8 + 16;
     cudaError_t e = allow_smem(reinterpret_cast<const void*>(project_tc_kernel), (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = std::min(a.n_tiles, sm_count());

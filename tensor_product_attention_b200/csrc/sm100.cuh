@@ -73,6 +73,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
     return false;
 }
 
+// Polls granted to the end-of-kernel drains (copies and MMAs still in flight).  Kept
+// apart from the run-time wait limit, so that a lowered limit can never let a CTA
+// exit while its own copies or MMAs are still landing.
+constexpr uint32_t kDrainLimit = 1u << 24;
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kDrainLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return;
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
