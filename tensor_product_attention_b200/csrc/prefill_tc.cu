@@ -17,16 +17,19 @@
 // q~) instead of once per (query, key) pair: the same sums, reassociated.
 //
 // One CTA = 256 rows (two 128-row M-blocks: 256/h queries x h heads) of one sequence,
-// walking key tiles of KT = 128/R keys.  Warp roles:
+// walking key tiles of KT = 64/R keys (64 U columns).  Warp roles:
 //   warp 0     TMA: b^K, b^V tiles (2-D maps over the cache, 128-byte swizzle) and
 //              a^K, a^V tiles (bulk copies) into a ring of stages
-//   warp 1     TMEM owner (512 columns) and MMA issuer; the two M-blocks ping-pong so
-//              that one block's softmax overlaps the other block's MMAs
+//   warps 1-2  MMA issuers, one per M-block (warp 1 also owns the 512 TMEM columns):
+//              QK of tile t is issued before the PV of tile t-1, so a block's scores
+//              for the next tile are ready while its softmax still works on the current
+//              one.  A thread that polls an mbarrier stalls until its own MMAs have
+//              completed, so a single issuer would serialise the blocks; two overlap.
 //   warps 4-11 softmax for M-block 0 (warps 4-7) and 1 (warps 8-11), one row per thread
 // The control warpgroup (warps 0-3) hands registers to the softmax warpgroups with
 // setmaxnreg once the prologue is done.
-// TMEM: U_0 [0,128), U_1 [128,256), O_0 and O_1 after 256 (d_h columns each); W_b
-// overwrites the first half of U_b once the scores are read (bf16 pairs).
+// TMEM: U double-buffered per M-block, U_{b,x} at 64*(2b+x); O_b at 256 + b*d_h.  W
+// overwrites the first half of U_{b,x} once the scores are read (bf16 pairs).
 #include <algorithm>
 #include <cmath>
 
@@ -41,8 +44,13 @@ using namespace sm100;
 
 constexpr int kThreads = 384;   // 3 warpgroups: TMA/MMA, softmax block 0, softmax block 1
 constexpr int kRegsCtl = 96, kRegsSoftmax = 200;   // 128*96 + 256*200 = 63488 <= 384*168 (launch)
-constexpr uint32_t kBox = 128 * 128;        // one TMA box: 128 rows x 128 bytes
+constexpr int kUW = 64;                     // U columns per tile (= KT * R rows of b^K)
+constexpr uint32_t kBox = kUW * 128;        // one TMA box: 64 rows x 128 bytes
 constexpr float kRescale = 8.f;             // lazy rescale threshold (log2 units)
+// a^K, a^V tiles transposed to one row per head (R = 2, h = 16): a row holds the tile's
+// 32 keys x (2 bf16) = 128 bytes, padded to 144 so that 16 heads spread over the banks
+constexpr int kATS = 2;                     // transposed tiles in flight
+constexpr uint32_t kATPitch = 144;
 
 struct PrefillTcArgs {
     const __nv_bfloat16* a_q;     // [T][H][Rq]
@@ -76,10 +84,10 @@ __device__ __forceinline__ void load_r(const __nv_bfloat16* base, int idx, float
 // reference max m_ref: d_j = sum_s a^K_{j,h,s} U_{(j,s)} - m_ref (log2 units), mx =
 // max_j d_j, p_j = 2^d_j, lsum = sum_j p_j, and the W row (p_j a^V_{j,h,s}) in K order
 // (j, s) packed as bf16 pairs.  MASKED applies the causal bound j <= p_i (diagonal tiles).
-template <int R, bool MASKED, int HS_>
+template <int R, bool MASKED, int HS_, bool AT = false>
 __device__ __forceinline__ void softmax_pass(uint32_t u_addr, const __nv_bfloat16* ak,
                                              const __nv_bfloat16* av, int H, int h, int j0, int p_i,
-                                             float m_ref, float& mx, float& lsum, uint32_t (&wp)[64]) {
+                                             float m_ref, float& mx, float& lsum, uint32_t (&wp)[32]) {
     const int HS = HS_ > 0 ? HS_ : H;   // head count, compile-time when known
     mx = -INFINITY;
     lsum = 0.f;
@@ -90,16 +98,28 @@ __device__ __forceinline__ void softmax_pass(uint32_t u_addr, const __nv_bfloat1
         const uint32_t* avr = reinterpret_cast<const uint32_t*>(av) + h;
         float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         float lsa[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
+        {
+            constexpr int hf = 0;
             uint32_t u[64];
-            tmem_ld32(u_addr + (uint32_t)hf * 64u, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-            tmem_ld32(u_addr + (uint32_t)hf * 64u + 32u, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+            tmem_ld32(u_addr, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+            tmem_ld32(u_addr + 32u, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
             uint32_t wa[32], wv[32];
+            if constexpr (AT) {
+                // ak, av point at this head's transposed rows: 4 keys per 16-byte load
+                const uint4* k4 = reinterpret_cast<const uint4*>(ak);
+                const uint4* v4 = reinterpret_cast<const uint4*>(av);
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                wa[q] = akr[(hf * 32 + q) * HS];
-                wv[q] = avr[(hf * 32 + q) * HS];
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 x = k4[c], y = v4[c];
+                    wa[4 * c] = x.x; wa[4 * c + 1] = x.y; wa[4 * c + 2] = x.z; wa[4 * c + 3] = x.w;
+                    wv[4 * c] = y.x; wv[4 * c + 1] = y.y; wv[4 * c + 2] = y.z; wv[4 * c + 3] = y.w;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    wa[q] = akr[q * HS];
+                    wv[q] = avr[q * HS];
+                }
             }
             tmem_ld_wait();
 #pragma unroll
@@ -124,11 +144,11 @@ __device__ __forceinline__ void softmax_pass(uint32_t u_addr, const __nv_bfloat1
     }
     constexpr int KPH = 64 / R;          // keys per 64 U columns
     float wprev = 0.f;
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
+    {
+        constexpr int hf = 0;
         uint32_t u[64];
-        tmem_ld32(u_addr + (uint32_t)hf * 64u, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-        tmem_ld32(u_addr + (uint32_t)hf * 64u + 32u, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+        tmem_ld32(u_addr, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+        tmem_ld32(u_addr + 32u, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
         tmem_ld_wait();
 #pragma unroll
         for (int q = 0; q < KPH; ++q) {
@@ -159,24 +179,34 @@ template <int DH, int R, int HC>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                   const PrefillTcArgs a, const SeqParams start) {
-    constexpr int KT = 128 / R;            // keys per tile
+    constexpr int KT = kUW / R;            // keys per tile
     constexpr int NB = DH / 64;            // 64-wide column blocks of d_h
-    constexpr uint32_t kQBytes = NB * 256u * 128u;
-    constexpr int UW = KT * R;             // U columns per M-block (= 128)
+    // d_h = 64: q~ lives in TMEM (columns 384.., bf16 pairs) and QK reads it from there;
+    // d_h = 128 leaves no TMEM for it, so q~ stays in shared memory
+    constexpr bool QT = DH == 64;
+    constexpr uint32_t kQCol = 256u + 2u * DH;
+    constexpr uint32_t kQBytes = QT ? 0u : NB * 256u * 128u;
+    constexpr int UW = kUW;                // U columns per tile and M-block
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* sq = smem;                                   // q~, [NB][256 rows][128 B]
     uint8_t* stg = smem + kQBytes;                        // stages
-    uint64_t* bars = reinterpret_cast<uint64_t*>(stg + (size_t)a.stages * a.stage_bytes);
+    // R = 2 at h = 16: warp 3 transposes each tile's a^K, a^V into kATS row-per-head buffers
+    constexpr bool AT = R == 2 && HC == 16;
+    constexpr uint32_t kATBytes = AT ? 2u * HC * kATPitch : 0u;       // one transposed tile pair
+    uint8_t* atr = stg + (size_t)a.stages * a.stage_bytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(atr + kATS * kATBytes);
     uint64_t* kv_full = bars;
     uint64_t* kv_empty = kv_full + a.stages;
-    uint64_t* u_ready = kv_empty + a.stages;    // [2]
-    uint64_t* w_ready = u_ready + 2;            // [2]
-    uint64_t* o_done = w_ready + 2;             // [2]
-    uint64_t* fin = o_done + 2;                 // MMAs in flight at exit
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+    uint64_t* u_ready = kv_empty + a.stages;    // [2 blocks][2 buffers] scores in U
+    uint64_t* w_ready = u_ready + 4;            // [2][2] W written over U
+    uint64_t* o_ready = w_ready + 4;            // [2] a PV into O_b has completed
+    uint64_t* o_done = o_ready + 2;             // [2] the last PV into O_b has completed
+    uint64_t* fin = o_done + 2;                 // [2] each issuer's MMAs in flight at exit
+    uint64_t* at_ready = fin + 2;               // [kATS] a transposed tile pair is written
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(at_ready + kATS);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -202,20 +232,32 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     };
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < a.stages; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
-        for (int i = 0; i < 2; ++i) {
+        // a stage is free once both M-blocks' issuers have committed their PV of it
+        for (int s = 0; s < a.stages; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 2); }
+        for (int i = 0; i < 4; ++i) {
             mbar_init(&u_ready[i], 1);
             mbar_init(&w_ready[i], 128);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&o_ready[i], 1);
             mbar_init(&o_done[i], 1);
         }
-        mbar_init(fin, 1);
+        mbar_init(&fin[0], 1);
+        mbar_init(&fin[1], 1);
+        for (int i = 0; i < kATS; ++i) mbar_init(&at_ready[i], 32);
         *abort = 0;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) { prefetch_tensormap(&tmk); prefetch_tensormap(&tmv); }
     if (warp == 1) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
 
-    // ---- prologue: q~ rows (bf16, 128-byte swizzled K-major) by the 256 softmax threads
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // ---- prologue: q~ rows by the 256 softmax threads, into TMEM (QT) or into shared
+    // memory (bf16, 128-byte swizzled K-major)
     if (warp >= 4) {
         const int row = threadIdx.x - 128;                // 0..255
         const int i_loc = row / H, h = row - (row / H) * H;
@@ -224,7 +266,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         float aq[16];
         for (int r = 0; r < a.Rq; ++r) aq[r] = vq ? __bfloat162float(a.a_q[(t * H + h) * a.Rq + r]) * a.qscale : 0.f;
         const __nv_bfloat16* bq = a.b_q + t * a.Rq * DH;
-#pragma unroll 1
+        uint32_t qw[QT ? DH / 2 : 1];
+#pragma unroll
         for (int k8 = 0; k8 < DH; k8 += 8) {
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             if (vq) {
@@ -242,15 +285,24 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             uint4 w;
             w.x = pack_bf16(acc[0], acc[1]); w.y = pack_bf16(acc[2], acc[3]);
             w.z = pack_bf16(acc[4], acc[5]); w.w = pack_bf16(acc[6], acc[7]);
-            const int cb = k8 >> 6;
-            *reinterpret_cast<uint4*>(sq + cb * (256u * 128u) + sw128_offset(row, (k8 & 63) * 2)) = w;
+            if constexpr (QT) {
+                qw[k8 / 2] = w.x; qw[k8 / 2 + 1] = w.y; qw[k8 / 2 + 2] = w.z; qw[k8 / 2 + 3] = w.w;
+            } else {
+                const int cb = k8 >> 6;
+                *reinterpret_cast<uint4*>(sq + cb * (256u * 128u) + sw128_offset(row, (k8 & 63) * 2)) = w;
+            }
         }
-        fence_proxy_async_smem();
+        if constexpr (QT) {
+            const int bl = row >> 7;
+            tmem_st32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + kQCol + (uint32_t)bl * (DH / 2), qw);
+            tmem_st_wait();
+        } else {
+            fence_proxy_async_smem();
+        }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
     if (warp < 4) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
       if (warp == 0) {
@@ -283,59 +335,102 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     drain_wait(&kv_full[s], (uint32_t)((fills - 1) & 1));
             }
         }
-      } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+      } else if (warp <= 2) {
+        // ------------------------------------------------------------ MMA issuers
+        // Warp 1 issues every MMA of M-block 0, warp 2 those of M-block 1.  An issuing
+        // thread that polls an mbarrier waits there until its own MMAs in flight have
+        // completed; with one issuer per block, that wait overlaps the other block's MMAs.
         if (lane == 0) {
+            const int bl = warp - 1;
             const uint32_t idesc_qk = idesc_bf16(128, UW, 0, 0);
             const uint32_t idesc_pv = idesc_bf16(128, DH, 0, 1);
-            const uint32_t q_base = smem_u32(sq);
-            for (int t = 0; t <= n_tiles && !*abort; ++t) {
-                const int s = t % a.stages;
-                if (t < n_tiles) {
-                    if (!mbar_wait(&kv_full[s], (uint32_t)((t / a.stages) & 1), lim, a.err, abort)) break;
-                    tc_fence_after();
-                }
-                bool ok = true;
-                for (int bl = 0; bl < 2; ++bl) {
-                    const uint32_t u_col = tmem + (uint32_t)bl * 128u;
-                    const uint32_t o_col = tmem + 256u + (uint32_t)bl * DH;
-                    if (t > 0) {
-                        // O_bl += W_bl(t-1) . b^V(t-1)
-                        if (!mbar_wait(&w_ready[bl], (uint32_t)((t - 1) & 1), lim, a.err, abort)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const int sp = (t - 1) % a.stages;
-                        const uint32_t bv = smem_u32(stage_bv(sp));
+            const uint32_t q_base = smem_u32(sq) + (uint32_t)bl * 128u * 128u;
+            const uint32_t o_col = tmem + 256u + (uint32_t)bl * DH;
+            // U_{bl, t&1} = q~_bl . b^K(t)^T, b^K from stage st
+            auto issue_qk = [&](int t, int st) {
+                const uint32_t bk = smem_u32(stage_bk(st));
+                const uint32_t u_col = tmem + (uint32_t)(2 * bl + (t & 1)) * kUW;
 #pragma unroll
-                        for (int k = 0; k < UW / 16; ++k)
-                            mma_ts(o_col, u_col + (uint32_t)k * 8u,
-                                   smem_desc(bv + (uint32_t)k * 2048u, kBox, 1024, kSwizzle128),
-                                   idesc_pv, (t - 1 > 0 || k > 0) ? 1u : 0u);
-                        if (bl == 1) mma_commit(&kv_empty[sp]);
-                        if (t == n_tiles) mma_commit(&o_done[bl]);
-                    }
-                    if (t < n_tiles) {
-                        // U_bl = q~_bl . b^K(t)^T
-                        const uint32_t bk = smem_u32(stage_bk(s));
-#pragma unroll
-                        for (int k = 0; k < DH / 16; ++k) {
-                            const uint32_t cb = (uint32_t)(k >> 2), kk = (uint32_t)(k & 3) * 32u;
-                            mma_ss(u_col,
-                                   smem_desc(q_base + cb * 256u * 128u + (uint32_t)bl * 128u * 128u + kk,
-                                             16, 1024, kSwizzle128),
-                                   smem_desc(bk + cb * kBox + kk, 16, 1024, kSwizzle128), idesc_qk,
-                                   k > 0 ? 1u : 0u);
-                        }
-                        mma_commit(&u_ready[bl]);
-                    }
+                for (int k = 0; k < DH / 16; ++k) {
+                    const uint32_t cb = (uint32_t)(k >> 2), kk = (uint32_t)(k & 3) * 32u;
+                    const uint64_t bdesc = smem_desc(bk + cb * kBox + kk, 16, 1024, kSwizzle128);
+                    if constexpr (QT)
+                        mma_ts(u_col, tmem + kQCol + (uint32_t)bl * (DH / 2) + (uint32_t)k * 8u, bdesc, idesc_qk,
+                               k > 0 ? 1u : 0u);
+                    else
+                        mma_ss(u_col, smem_desc(q_base + cb * 256u * 128u + kk, 16, 1024, kSwizzle128), bdesc,
+                               idesc_qk, k > 0 ? 1u : 0u);
                 }
-                if (!ok) break;
+                mma_commit(&u_ready[2 * bl + (t & 1)]);
+            };
+            // every poll (and every shared-memory read) made by this thread waits for its
+            // MMAs in flight, so the loop keeps them to the one wait it needs per tile
+            bool ok = mbar_wait(&kv_full[0], 0u, lim, a.err, abort);
+            if (ok) { tc_fence_after(); issue_qk(0, 0); }
+            if (ok && n_tiles > 1 && (ok = mbar_wait(&kv_full[1], 0u, lim, a.err, abort))) {
+                tc_fence_after();
+                issue_qk(1, 1);
             }
-            // every MMA issued has completed before TMEM is released
-            mma_commit(fin);
-            drain_wait(fin, 0);
+            // Steady state: one wait for W(t), then PV(t) and QK(t+2) back to back.
+            // QK(t+2) overwrites U_{bl, t&1} after PV(t) has read W from it (one issuer,
+            // in order).  s0 = stage of tile t; s2, ph2 = stage and parity of tile t+2.
+            int s0 = 0, s2 = 2;
+            uint32_t ph2 = 0;
+            for (int t = 0; ok && t < n_tiles; ++t) {
+                if (!mbar_wait(&w_ready[2 * bl + (t & 1)], (uint32_t)((t >> 1) & 1), lim, a.err, abort)) break;
+                // block 0's softmax clears the b^V rows past the valid keys of the last
+                // tile before it hands over its W; block 1's PV reads the same stage
+                if (bl == 1 && t == n_tiles - 1 && t * KT + KT > kv_len &&
+                    !mbar_wait(&w_ready[t & 1], (uint32_t)((t >> 1) & 1), lim, a.err, abort))
+                    break;
+                const bool next = t + 2 < n_tiles;
+                if (next && !mbar_wait(&kv_full[s2], ph2, lim, a.err, abort)) break;
+                tc_fence_after();
+                // O_bl += W_bl(t) . b^V(t)
+                const uint32_t bv = smem_u32(stage_bv(s0));
+                const uint32_t w_col = tmem + (uint32_t)(2 * bl + (t & 1)) * kUW;
+#pragma unroll
+                for (int k = 0; k < UW / 16; ++k)
+                    mma_ts(o_col, w_col + (uint32_t)k * 8u, smem_desc(bv + (uint32_t)k * 2048u, kBox, 1024, kSwizzle128),
+                           idesc_pv, (t > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&o_ready[bl]);
+                if (t == n_tiles - 1) mma_commit(&o_done[bl]);
+                mma_commit(&kv_empty[s0]);
+                if (next) issue_qk(t + 2, s2);
+                s0 = s0 + 1 == a.stages ? 0 : s0 + 1;
+                if (++s2 == a.stages) { s2 = 0; ph2 ^= 1u; }
+            }
+            // every MMA this thread issued has completed before TMEM is released
+            mma_commit(&fin[bl]);
+            drain_wait(&fin[bl], 0);
+        }
+      } else if constexpr (AT) {
+        // ------------------------------------------------------------ a-tile transpose
+        // warp 3: a^K, a^V of tile t from [key][head] pairs to one row per head, into
+        // buffer t % kATS once both M-blocks' softmax have finished tile t - kATS
+        constexpr int kWords = KT * HC;                  // (key, head) pairs per tile
+        int s = 0;
+        uint32_t ph = 0;
+        for (int t = 0; t < n_tiles; ++t) {
+            bool good = mbar_wait(&kv_full[s], ph, lim, a.err, abort);
+            if (good && t >= kATS) {
+                const int tp = t - kATS;
+                good = mbar_wait(&w_ready[tp & 1], (uint32_t)((tp >> 1) & 1), lim, a.err, abort) &&
+                       mbar_wait(&w_ready[2 + (tp & 1)], (uint32_t)((tp >> 1) & 1), lim, a.err, abort);
+            }
+            if (__any_sync(0xffffffffu, !good)) break;
+            const uint32_t* sk = reinterpret_cast<const uint32_t*>(stage_ak(s));
+            const uint32_t* sv = reinterpret_cast<const uint32_t*>(stage_av(s));
+            uint32_t* dk = reinterpret_cast<uint32_t*>(atr + (t % kATS) * kATBytes);
+            uint32_t* dv = dk + HC * (kATPitch / 4);
+#pragma unroll 4
+            for (int w = lane; w < kWords; w += 32) {
+                const int j = w / HC, hh = w % HC;
+                dk[hh * (kATPitch / 4) + j] = sk[w];
+                dv[hh * (kATPitch / 4) + j] = sv[w];
+            }
+            mbar_arrive(&at_ready[t % kATS]);
+            if (++s == a.stages) { s = 0; ph ^= 1u; }
         }
       }
     } else {
@@ -349,28 +444,36 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         const bool vq = i_loc < nq;
         const int p_i = p0 + min(i_loc, nq - 1);
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-        const uint32_t u_col = (uint32_t)bl * 128u;
         const uint32_t o_col = 256u + (uint32_t)bl * DH;
         float m_use = -INFINITY, l = 0.f;
         bool alive = true;
-        const uint32_t u_addr = lane_addr + u_col;
         for (int t = 0; t < n_tiles; ++t) {
+            const int ub = 2 * bl + (t & 1);
             // leave together: the warp votes below need every lane
-            const bool got = mbar_wait(&u_ready[bl], (uint32_t)(t & 1), lim, a.err, abort);
+            bool got = mbar_wait(&u_ready[ub], (uint32_t)((t >> 1) & 1), lim, a.err, abort);
+            if constexpr (AT) got = got && mbar_wait(&at_ready[t % kATS], (uint32_t)((t / kATS) & 1), lim, a.err, abort);
             if (__any_sync(0xffffffffu, !got)) { alive = false; break; }
             tc_fence_after();
+            const uint32_t u_addr = lane_addr + (uint32_t)ub * kUW;
             const int s = t % a.stages;
             const int j0 = t * KT;
-            const __nv_bfloat16* ak = stage_ak(s);
-            const __nv_bfloat16* av = stage_av(s);
+            const __nv_bfloat16* ak;
+            const __nv_bfloat16* av;
+            if constexpr (AT) {
+                ak = reinterpret_cast<const __nv_bfloat16*>(atr + (t % kATS) * kATBytes + h * kATPitch);
+                av = reinterpret_cast<const __nv_bfloat16*>(atr + (t % kATS) * kATBytes + (HC + h) * kATPitch);
+            } else {
+                ak = stage_ak(s);
+                av = stage_av(s);
+            }
             const bool masked = j0 + KT - 1 > p0;        // same for every row of the CTA
-            uint32_t wp[64];
+            uint32_t wp[32];
             float mx = -INFINITY, lsum = 0.f;
             bool ok = false;
             if (t > 0) {
                 // common case: one pass against the running max
-                if (masked) softmax_pass<R, true, HC>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
-                else softmax_pass<R, false, HC>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
+                if (masked) softmax_pass<R, true, HC, AT>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
+                else softmax_pass<R, false, HC, AT>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
                 ok = mx <= kRescale;
             }
             if (__all_sync(0xffffffffu, ok)) {
@@ -378,14 +481,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             } else {
                 // first tile, or the max rose by more than 2^kRescale: exact max, rescale O
                 if (t == 0) {
-                    if (masked) softmax_pass<R, true, HC>(u_addr, ak, av, H, h, j0, p_i, 0.f, mx, lsum, wp);
-                    else softmax_pass<R, false, HC>(u_addr, ak, av, H, h, j0, p_i, 0.f, mx, lsum, wp);
+                    if (masked) softmax_pass<R, true, HC, AT>(u_addr, ak, av, H, h, j0, p_i, 0.f, mx, lsum, wp);
+                    else softmax_pass<R, false, HC, AT>(u_addr, ak, av, H, h, j0, p_i, 0.f, mx, lsum, wp);
                 }
                 const float m_new = (t == 0) ? mx : (mx > kRescale ? m_use + mx : m_use);
                 const float alpha = (t == 0) ? 1.f : ex2(m_use - m_new);
                 if (t > 0) l *= alpha;
                 if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-                    // O row *= alpha (PV(t-1) has completed: QK(t) was committed after it)
+                    // O row *= alpha, once PV(t-1) into O has completed
+                    const bool pv_done = mbar_wait(&o_ready[bl], (uint32_t)((t - 1) & 1), lim, a.err, abort);
+                    if (__any_sync(0xffffffffu, !pv_done)) { alive = false; break; }
+                    tc_fence_after();
 #pragma unroll
                     for (int c = 0; c < DH / 32; ++c) {
                         uint32_t o[32];
@@ -398,20 +504,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     tmem_st_wait();
                 }
                 m_use = m_new;
-                if (masked) softmax_pass<R, true, HC>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
-                else softmax_pass<R, false, HC>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
+                if (masked) softmax_pass<R, true, HC, AT>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
+                else softmax_pass<R, false, HC, AT>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
                 l += lsum;
             }
             // W over the first half of U (the scores have all been read)
-            tmem_st32(u_addr, *reinterpret_cast<uint32_t(*)[32]>(&wp[0]));
-            tmem_st32(u_addr + 32u, *reinterpret_cast<uint32_t(*)[32]>(&wp[32]));
+            tmem_st32(u_addr, wp);
             tmem_st_wait();
             if (bl == 0 && t == n_tiles - 1 && j0 + KT > kv_len) {
                 // keys at or past the valid length: clear their b^V rows so that
                 // 0 * (whatever the cache holds there) stays 0 in the PV product
                 uint8_t* bv = stage_bv(s);
                 const int first = (kv_len - j0) * R;
-                for (int rr = first + (threadIdx.x - 128); rr < 128; rr += 128)
+                for (int rr = first + (threadIdx.x - 128); rr < UW; rr += 128)
                     for (int cb = 0; cb < NB; ++cb) {
                         uint4* pz = reinterpret_cast<uint4*>(bv + cb * kBox + rr * 128);
 #pragma unroll
@@ -420,10 +525,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 fence_proxy_async_smem();
             }
             tc_fence_before();
-            mbar_arrive(&w_ready[bl]);
+            mbar_arrive(&w_ready[ub]);
         }
-        const bool fin = alive && mbar_wait(&o_done[bl], 0u, lim, a.err, abort);
-        if (__all_sync(0xffffffffu, fin)) {
+        const bool done_ok = alive && mbar_wait(&o_done[bl], 0u, lim, a.err, abort);
+        if (__all_sync(0xffffffffu, done_ok)) {
             tc_fence_after();
             const float inv = a.out_scale / l;
             const long long t = (long long)b * a.S + q0 + i_loc;
@@ -459,22 +564,23 @@ template <int DH, int R, int HC>
 cudaError_t launch_t(const PrefillTcArgs& a0, const tpa_cache& c, int batch, const SeqParams& start,
                      cudaStream_t st) {
     PrefillTcArgs a = a0;
-    constexpr int KT = 128 / R;
+    constexpr int KT = kUW / R;
     constexpr int NB = DH / 64;
     a.a_bytes = (uint32_t)(KT * a.H * R * 2);
     const uint32_t a_pad = (a.a_bytes + 127u) & ~127u;
     a.stage_bytes = ((2u * NB * kBox + 2u * a_pad) + 1023u) & ~1023u;
-    const uint32_t q_bytes = NB * 256u * 128u;
-    const uint32_t budget = 227u * 1024u - 1024u - 256u - q_bytes;
-    a.stages = std::min(4, (int)(budget / a.stage_bytes));
-    if (a.stages < 2) return cudaErrorInvalidValue;
+    const uint32_t q_bytes = DH == 64 ? 0u : NB * 256u * 128u;   // q~ in TMEM at d_h 64
+    const uint32_t at_bytes = (R == 2 && HC == 16) ? kATS * 2u * HC * kATPitch : 0u;
+    const uint32_t budget = 227u * 1024u - 1024u - 512u - q_bytes - at_bytes;
+    a.stages = std::min(8, (int)(budget / a.stage_bytes));
+    if (a.stages < 3) return cudaErrorInvalidValue;   // QK(t+2) and PV(t) use different stages
     CUtensorMap tmk, tmv;
     const uint64_t dims[2] = {(uint64_t)DH, (uint64_t)c.batch * c.capacity * R};
     const uint64_t stride[1] = {(uint64_t)DH * 2};
-    const uint32_t box[2] = {64, 128};
+    const uint32_t box[2] = {64, (uint32_t)kUW};
     if (!make_tmap_bf16(&tmk, c.b_k, 2, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 2, dims, stride, box))
         return cudaErrorInvalidValue;
-    const size_t smem = 1024 + q_bytes + (size_t)a.stages * a.stage_bytes + (2 * a.stages + 7) * 8 + 16;
+    const size_t smem = 1024 + q_bytes + (size_t)a.stages * a.stage_bytes + at_bytes + (2 * a.stages + 14 + kATS) * 8 + 16;
     cudaError_t e = allow_smem(reinterpret_cast<const void*>(prefill_tc_kernel<DH, R, HC>), (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.n_qblocks, batch);
@@ -490,7 +596,12 @@ bool prefill_tc_supported(const Shape& s) {
     if (s.H < 1 || 128 % s.H != 0) return false;
     if ((s.H * s.Rk) % 8 != 0) return false;          // 16-byte bulk copies of a^K / a^V rows
     if (s.Rq < 1 || s.Rq > 16) return false;
-    return true;
+    // at least three stages of (b^K, b^V boxes + a^K, a^V tiles of 128*h bytes) beside q~
+    const uint32_t nb = (uint32_t)s.Dh / 64u;
+    const uint32_t a_pad = (128u * (uint32_t)s.H + 127u) & ~127u;
+    const uint32_t stage = ((2u * nb * kBox + 2u * a_pad) + 1023u) & ~1023u;
+    const uint32_t at_bytes = (s.Rk == 2 && s.H == 16) ? kATS * 2u * 16u * kATPitch : 0u;
+    return 227u * 1024u - 1024u - 512u - nb * 256u * 128u - at_bytes >= 3u * stage;
 }
 
 cudaError_t launch_prefill_tc(const Shape& s, const tpa_factors& q, const tpa_cache& c, int batch,
