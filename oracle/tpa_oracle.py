@@ -55,13 +55,18 @@ class Dims:
 
 def factor_widths(dims: Dims) -> dict:
     """Output width of each of the six bias-free projections ([review] 类定义与初始化):
-    W_A_* map d_model -> n_heads*rank, W_B_* map d_model -> rank*head_dim."""
+    W_A_* map d_model -> n_heads*rank, W_B_* map d_model -> rank*head_dim.
+
+    TPA-KVonly (rank_q = 0) keeps the standard query projection ([review] 实验/结果
+    names the variant; its projection is not printed).  Reading taken: it takes the
+    b_q slot as W_Q with n_heads*head_dim outputs, viewed (n_heads, head_dim), and the
+    a_q slot is empty."""
     h, d = dims.n_heads, dims.head_dim
     return {
         "a_q": h * dims.rank_q,
         "a_k": h * dims.rank_k,
         "a_v": h * dims.rank_v,
-        "b_q": dims.rank_q * d,
+        "b_q": (dims.rank_q if dims.rank_q > 0 else h) * d,
         "b_k": dims.rank_k * d,
         "b_v": dims.rank_v * d,
     }
@@ -122,7 +127,8 @@ def split_factors(y: np.ndarray, dims: Dims) -> dict:
     """Cut the concatenated projection output into the six factors, with the views of
     [review] 前向传播: A_* is viewed (.., n_heads, rank) and B_* (.., rank, head_dim),
     so column h*R + r of W_A_* is (head h, rank r) and column r*d + k of W_B_* is
-    (rank r, dim k).  The concatenation order is FACTOR_NAMES."""
+    (rank r, dim k).  The concatenation order is FACTOR_NAMES.  For TPA-KVonly the
+    result holds the query ``q`` (.., n_heads, head_dim) in place of a_q and b_q."""
     widths = factor_widths(dims)
     h, d = dims.n_heads, dims.head_dim
     ranks = {"q": dims.rank_q, "k": dims.rank_k, "v": dims.rank_v}
@@ -133,7 +139,10 @@ def split_factors(y: np.ndarray, dims: Dims) -> dict:
         w = widths[name]
         part = y[..., col:col + w]
         r = ranks[name[-1]]
-        if name.startswith("a_"):
+        if dims.rank_q == 0 and name in ("a_q", "b_q"):
+            if name == "b_q":
+                out["q"] = part.reshape(lead + (h, d))     # TPA-KVonly: the plain query
+        elif name.startswith("a_"):
             out[name] = part.reshape(lead + (h, r))
         else:
             out[name] = part.reshape(lead + (r, d))
@@ -211,8 +220,6 @@ def tpa_forward(x: np.ndarray, w_cat: np.ndarray, dims: Dims, rope_base: float,
     x: [B, S, d_model].  Returns (out [B, S, h, d], new) where ``new`` holds the
     un-rotated factors of the S new tokens ([B, S, ...] each).
     """
-    if dims.rank_q == 0:
-        raise ValueError("tpa_forward projects factorised queries; rank_q must be > 0")
     x = np.asarray(x, dtype=np.float64)
     B, S, _ = x.shape
     new = project(x.reshape(B * S, -1), w_cat, dims)
@@ -224,7 +231,10 @@ def tpa_forward(x: np.ndarray, w_cat: np.ndarray, dims: Dims, rope_base: float,
             head = prior[n][b][:start_pos] if (prior is not None and start_pos) else \
                 np.zeros((0,) + new[n].shape[2:])
             cache[n] = np.concatenate([np.asarray(head, np.float64), new[n][b]], axis=0)
-        q = materialize(new["a_q"][b], new["b_q"][b], dims.rank_q)
+        if dims.rank_q == 0:
+            q = new["q"][b]                               # TPA-KVonly: plain query
+        else:
+            q = materialize(new["a_q"][b], new["b_q"][b], dims.rank_q)
         k = materialize(cache["a_k"], cache["b_k"], dims.rank_k)
         v = materialize(cache["a_v"], cache["b_v"], dims.rank_v)
         q_pos = start_pos + np.arange(S)
@@ -304,7 +314,10 @@ def tpa_forward_rows(x: np.ndarray, w_cat: np.ndarray, dims: Dims, rope_base: fl
     x = np.asarray(x, dtype=np.float64)
     rows = np.asarray(rows).reshape(-1)
     f = project(x, w_cat, dims)
-    q = materialize(f["a_q"][rows], f["b_q"][rows], dims.rank_q)
+    if dims.rank_q == 0:
+        q = f["q"][rows]                                  # TPA-KVonly: plain query
+    else:
+        q = materialize(f["a_q"][rows], f["b_q"][rows], dims.rank_q)
     k = materialize(f["a_k"], f["b_k"], dims.rank_k)
     v = materialize(f["a_v"], f["b_v"], dims.rank_v)
     q = rope_rotate(q, rows, rope_base)

@@ -401,3 +401,65 @@ def test_forward_rows_equals_forward():
     full, _ = oracle.tpa_forward(x, w, dims, 1e4)
     rows = [0, 5, 20]
     assert rel(oracle.tpa_forward_rows(x[0], w, dims, 1e4, rows), full[0, rows]) < 1e-13
+
+
+# ------------------------------------------------------------------- TPA-KVonly
+
+def _kvonly_weights(g, dims):
+    widths = oracle.factor_widths(dims)
+    assert widths["a_q"] == 0 and widths["b_q"] == dims.n_heads * dims.head_dim
+    ws = {n: g.standard_normal((widths[n], dims.d_model)) / math.sqrt(dims.d_model) for n in oracle.FACTOR_NAMES}
+    return ws, np.concatenate([ws[n] for n in oracle.FACTOR_NAMES], axis=0)
+
+
+def test_kvonly_projection_is_a_plain_query_linear_plus_kv_factors():
+    # TPA-KVonly ([review] 实验/结果): the query is a standard per-head linear map.
+    g = gen(21)
+    dims = Dims(d_model=24, n_heads=3, head_dim=8, rank_q=0, rank_k=2, rank_v=3)
+    T = 7
+    x = g.standard_normal((T, dims.d_model))
+    ws, w_cat = _kvonly_weights(g, dims)
+    got = oracle.project(x, w_cat, dims)
+    assert set(got) == {"q", "a_k", "a_v", "b_k", "b_v"}
+    xt = torch.from_numpy(x)
+    want_q = F.linear(xt, torch.from_numpy(ws["b_q"])).view(T, dims.n_heads, dims.head_dim).numpy()
+    assert rel(got["q"], want_q) < TOL
+    want_bv = F.linear(xt, torch.from_numpy(ws["b_v"])).view(T, dims.rank_v, dims.head_dim).numpy()
+    assert rel(got["b_v"], want_bv) < TOL
+
+
+def test_kvonly_forward_is_textbook_attention_on_rotated_q_and_materialised_kv():
+    # Independent route in torch: F.linear for the projections, bmm/R for K and V,
+    # RoPE as complex multiplication, causal fp64 scaled_dot_product_attention.
+    g = gen(22)
+    dims = Dims(d_model=20, n_heads=4, head_dim=8, rank_q=0, rank_k=2, rank_v=2)
+    B, S, base = 2, 11, 1e4
+    x = g.standard_normal((B, S, dims.d_model))
+    ws, w_cat = _kvonly_weights(g, dims)
+    out, new = oracle.tpa_forward(x, w_cat, dims, base)
+    h, d, R = dims.n_heads, dims.head_dim, dims.rank_k
+    theta = torch.tensor(base, dtype=torch.float64) ** (-(torch.arange(0, d, 2, dtype=torch.float64) / d))
+    pos = torch.arange(S, dtype=torch.float64)
+    rot = torch.polar(torch.ones(S, d // 2, dtype=torch.float64), pos[:, None] * theta[None, :])
+
+    def rope(t):                                   # t [S, h, d]
+        c = torch.view_as_complex(t.reshape(S, h, d // 2, 2).contiguous())
+        return torch.view_as_real(c * rot[:, None, :]).reshape(S, h, d)
+
+    for b in range(B):
+        xt = torch.from_numpy(x[b])
+        lin = {n: F.linear(xt, torch.from_numpy(ws[n])) for n in oracle.FACTOR_NAMES if ws[n].shape[0]}
+        q = lin["b_q"].view(S, h, d)
+        k = torch.bmm(lin["a_k"].view(S, h, R), lin["b_k"].view(S, R, d)) / R
+        v = torch.bmm(lin["a_v"].view(S, h, R), lin["b_v"].view(S, R, d)) / R
+        q, k = rope(q), rope(k)
+        want = F.scaled_dot_product_attention(q.permute(1, 0, 2), k.permute(1, 0, 2), v.permute(1, 0, 2),
+                                              is_causal=True).permute(1, 0, 2)
+        assert rel(out[b], want.numpy()) < 1e-12
+        # the pre-rotated form the kernels use: rotate q and B_K, then attend from factors
+        qf = {"q": oracle.rope_rotate(new["q"][b], np.arange(S), base)}
+        kv = {"a_k": new["a_k"][b], "a_v": new["a_v"][b], "b_v": new["b_v"][b],
+              "b_k": oracle.rope_rotate(new["b_k"][b], np.arange(S), base)}
+        assert rel(oracle.attend_from_factors(qf, kv, dims, np.arange(S)), out[b]) < 1e-12
+    rows = [0, 6, 10]
+    assert rel(oracle.tpa_forward_rows(x[1], w_cat, dims, base, rows), out[1, rows]) < 1e-12
