@@ -70,8 +70,8 @@ typedef enum tpa_dtype { TPA_F32 = 0, TPA_BF16 = 1 } tpa_dtype;
 
 /* Shape of one TPA layer: the page's ModelArgs (dim, n_heads, head_dim, q_rank, rank)
  * [review, 代码 类定义与初始化], with rank split into rank_k and rank_v.
- * rank_q = 0 selects TPA-KVonly: the query is a plain per-head vector [h][d_h]
- * (decode only in this version). */
+ * rank_q = 0 selects TPA-KVonly [review, 实验/结果]: the query is a plain per-head
+ * vector [h][d_h] held in the b_q slot; a_q is unused. */
 typedef struct tpa_dims {
     int32_t d_model;
     int32_t n_heads;     /* h */
@@ -84,7 +84,8 @@ typedef struct tpa_dims {
 
 /* The six factor tensors of T tokens (device):
  *   a_q [T][h][R_Q]   a_k [T][h][R_K]   a_v [T][h][R_V]
- *   b_q [T][R_Q][d_h] b_k [T][R_K][d_h] b_v [T][R_V][d_h]   (b_q, b_k rotated) */
+ *   b_q [T][R_Q][d_h] b_k [T][R_K][d_h] b_v [T][R_V][d_h]   (b_q, b_k rotated)
+ * TPA-KVonly (rank_q = 0): b_q holds the rotated query [T][h][d_h]; a_q may be NULL. */
 typedef struct tpa_factors {
     void* a_q; void* b_q;
     void* a_k; void* b_k;
@@ -129,7 +130,11 @@ tpa_status tpa_rope_table(const tpa_dims* dims, double base, int32_t max_pos,
  *   start_pos host [batch]; every start_pos[b] + seqlen <= max_pos (else TPA_ERR_CAPACITY)
  *   rope_cs device table from tpa_rope_table with the same head_dim and >= max_pos rows
  *   out    device factor buffers for T tokens (all six set, none aliasing x or w_cat)
- * rank_q = 0 is TPA_ERR_UNSUPPORTED. */
+ * TPA-KVonly (rank_q = 0): the W_A_q block is empty and the W_B_q block is the plain
+ * query projection W_Q with h*d_h rows (row h*d_h + k is head h, dim k), so N =
+ * h(R_K+R_V) + d_h(h+R_K+R_V); out->b_q receives the rotated query [T][h][d_h] and
+ * out->a_q may be NULL.  The pages do not print this variant's projection; this
+ * layout is the reading taken. */
 tpa_status tpa_project(const tpa_dims* dims, const void* x, const void* w_cat,
                        int32_t batch, int32_t seqlen, const int32_t* start_pos,
                        const float* rope_cs, int32_t max_pos,
@@ -151,7 +156,8 @@ tpa_status tpa_cache_append(const tpa_dims* dims, const tpa_cache* cache,
  *   out[b*seqlen+i][h][:] = sum_j softmax_j(q_h . k_{j,h} / sqrt(d_h)) v_{j,h}
  * with q, k, v the (1/R) rank sums of the factors [review, §3 公式描述 and 前向传播;
  * jieyibu.net page, Ⅱ.1], evaluated from the factors without writing K or V out.
- *   q      device a_q, b_q (rotated) for batch*seqlen tokens (other members ignored)
+ *   q      device a_q, b_q (rotated) for batch*seqlen tokens (other members ignored);
+ *          TPA-KVonly: b_q = the rotated query [T][h][d_h], a_q ignored
  *   cache  must already hold positions 0 .. start_pos[b]+seqlen-1 of each sequence
  *   start_pos host [batch]
  *   out    device [batch*seqlen][h][d_h] */

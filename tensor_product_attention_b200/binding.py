@@ -160,6 +160,9 @@ def alloc_factors(dims: Dims, T: int, device="cuda", queries=True, kv=True) -> F
     if queries and dims.rank_q > 0:
         f.a_q = torch.empty((T, h, dims.rank_q), dtype=dt, device=device)
         f.b_q = torch.empty((T, dims.rank_q, d), dtype=dt, device=device)
+    elif queries:
+        # TPA-KVonly: the plain per-head query sits in the b_q slot, [T][h][d_h]
+        f.b_q = torch.empty((T, h, d), dtype=dt, device=device)
     if kv:
         f.a_k = torch.empty((T, h, dims.rank_k), dtype=dt, device=device)
         f.b_k = torch.empty((T, dims.rank_k, d), dtype=dt, device=device)

@@ -37,13 +37,16 @@ __global__ void __launch_bounds__(128) prefill_simt_kernel(PrefillArgs a, SeqPar
     const T* bk = reinterpret_cast<const T*>(a.cb_k);
     const T* bv = reinterpret_cast<const T*>(a.cb_v);
 
-    const float qscale = kLog2e / ((float)a.Rq * (float)a.Rk * sqrtf((float)a.Dh));
+    // TPA-KVonly (Rq = 0): the query row is given, q_{t,h} = b_q[t][h][:]
+    const float qscale = kLog2e / ((float)(a.Rq > 0 ? a.Rq : 1) * (float)a.Rk * sqrtf((float)a.Dh));
     float q[MAXU], acc[MAXU];
 #pragma unroll
     for (int u = 0; u < MAXU; ++u) {
         int e = lane + 32 * u;
         float v = 0.f;
         if (e < a.Dh)
+            if (a.Rq == 0)
+                v = to_f(bq[((long long)t * a.H + h) * a.Dh + e]);
             for (int r = 0; r < a.Rq; ++r)
                 v = fmaf(to_f(aq[((long long)t * a.H + h) * a.Rq + r]),
                          to_f(bq[((long long)t * a.Rq + r) * a.Dh + e]), v);

@@ -263,15 +263,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         const int i_loc = row / H, h = row - (row / H) * H;
         const bool vq = i_loc < nq;
         const long long t = (long long)b * a.S + q0 + (vq ? i_loc : 0);
+        // q~ = qscale * sum_r a^Q_r b^Q_r; TPA-KVonly (Rq = 0): qscale * q[t][h][:]
+        const int nr = a.Rq > 0 ? a.Rq : 1;
         float aq[16];
         for (int r = 0; r < a.Rq; ++r) aq[r] = vq ? __bfloat162float(a.a_q[(t * H + h) * a.Rq + r]) * a.qscale : 0.f;
-        const __nv_bfloat16* bq = a.b_q + t * a.Rq * DH;
+        if (a.Rq == 0) aq[0] = vq ? a.qscale : 0.f;
+        const __nv_bfloat16* bq = a.Rq > 0 ? a.b_q + t * a.Rq * DH : a.b_q + (t * H + h) * DH;
         uint32_t qw[QT ? DH / 2 : 1];
 #pragma unroll
         for (int k8 = 0; k8 < DH; k8 += 8) {
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             if (vq) {
-                for (int r = 0; r < a.Rq; ++r) {
+                for (int r = 0; r < nr; ++r) {
                     const uint4 raw = *reinterpret_cast<const uint4*>(bq + r * DH + k8);
                     const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
@@ -595,7 +598,7 @@ bool prefill_tc_supported(const Shape& s) {
     if (s.Rk != s.Rv || (s.Rk != 1 && s.Rk != 2 && s.Rk != 4)) return false;
     if (s.H < 1 || 128 % s.H != 0) return false;
     if ((s.H * s.Rk) % 8 != 0) return false;          // 16-byte bulk copies of a^K / a^V rows
-    if (s.Rq < 1 || s.Rq > 16) return false;
+    if (s.Rq < 0 || s.Rq > 16) return false;          // 0: TPA-KVonly, the query is given
     // at least three stages of (b^K, b^V boxes + a^K, a^V tiles of 128*h bytes) beside q~
     const uint32_t nb = (uint32_t)s.Dh / 64u;
     const uint32_t a_pad = (128u * (uint32_t)s.H + 127u) & ~127u;
@@ -620,7 +623,7 @@ cudaError_t launch_prefill_tc(const Shape& s, const tpa_factors& q, const tpa_ca
     a.cap = c.capacity;
     a.qpb = 256 / s.H;
     a.n_qblocks = (seqlen + a.qpb - 1) / a.qpb;
-    a.qscale = 1.4426950408889634f / ((float)s.Rq * (float)s.Rk * std::sqrt((float)s.Dh));
+    a.qscale = 1.4426950408889634f / ((float)(s.Rq > 0 ? s.Rq : 1) * (float)s.Rk * std::sqrt((float)s.Dh));
     a.out_scale = 1.f / (float)s.Rv;
     a.err = err;
     a.wait_limit = wait_limit;

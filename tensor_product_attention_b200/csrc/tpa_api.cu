@@ -111,11 +111,11 @@ tpa_status tpa_rope_table(const tpa_dims* d, double base, int32_t max_pos, float
 tpa_status tpa_project(const tpa_dims* d, const void* x, const void* w_cat, int32_t batch,
                        int32_t seqlen, const int32_t* start_pos, const float* rope_cs,
                        int32_t max_pos, const tpa_factors* out, tpa_stream_t stream) {
-    tpa_status st = check_dims(d, true);
+    tpa_status st = check_dims(d, false);
     if (st != TPA_OK) return st;
     if (d->d_model < 1) return TPA_ERR_INVALID;
     if (!x || !w_cat || !start_pos || !rope_cs || !out) return TPA_ERR_INVALID;
-    if (!out->a_q || !out->b_q || !out->a_k || !out->b_k || !out->a_v || !out->b_v)
+    if ((d->rank_q > 0 && !out->a_q) || !out->b_q || !out->a_k || !out->b_k || !out->a_v || !out->b_v)
         return TPA_ERR_INVALID;
     if (!aligned16(x) || !aligned16(w_cat) || !aligned16(rope_cs)) return TPA_ERR_INVALID;
     if (batch < 1 || batch > TPA_MAX_BATCH || seqlen < 1 || max_pos < 1)
@@ -163,11 +163,12 @@ tpa_status tpa_cache_append(const tpa_dims* d, const tpa_cache* c, const tpa_fac
 tpa_status tpa_prefill(const tpa_dims* d, const tpa_factors* q, const tpa_cache* c,
                        int32_t batch, int32_t seqlen, const int32_t* start_pos, void* out,
                        tpa_stream_t stream) {
-    tpa_status st = check_dims(d, true);
+    tpa_status st = check_dims(d, false);
     if (st != TPA_OK) return st;
     if ((st = check_cache(c, batch)) != TPA_OK) return st;
-    if (!q || !q->a_q || !q->b_q || !start_pos || !out) return TPA_ERR_INVALID;
-    if (!aligned16(q->a_q) || !aligned16(q->b_q) || !aligned16(out)) return TPA_ERR_INVALID;
+    if (!q || !q->b_q || !start_pos || !out) return TPA_ERR_INVALID;
+    if (d->rank_q > 0 && (!q->a_q || !aligned16(q->a_q))) return TPA_ERR_INVALID;
+    if (!aligned16(q->b_q) || !aligned16(out)) return TPA_ERR_INVALID;
     if (seqlen < 1) return TPA_ERR_INVALID;
     if (d->head_dim > 256) return TPA_ERR_UNSUPPORTED;
     SeqParams sp;

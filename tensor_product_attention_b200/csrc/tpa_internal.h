@@ -26,6 +26,8 @@ inline Shape shape_of(const tpa_dims& d) {
 }
 
 // Column layout of the stacked projection output: [a_q | a_k | a_v | b_q | b_k | b_v].
+// TPA-KVonly (rank_q = 0): a_q is empty and the b_q segment is the plain query
+// projection, h rows of d_h ([T][h][d_h]), rotated like B_Q.
 struct ProjLayout {
     int off[7];    // segment starts, off[6] = N
     void* dst[6];  // a_q, a_k, a_v, b_q, b_k, b_v
@@ -33,7 +35,8 @@ struct ProjLayout {
 
 inline ProjLayout proj_layout(const Shape& s, const tpa_factors& f) {
     ProjLayout L;
-    int w[6] = {s.H * s.Rq, s.H * s.Rk, s.H * s.Rv, s.Rq * s.Dh, s.Rk * s.Dh, s.Rv * s.Dh};
+    const int q_rows = s.Rq > 0 ? s.Rq : s.H;
+    int w[6] = {s.H * s.Rq, s.H * s.Rk, s.H * s.Rv, q_rows * s.Dh, s.Rk * s.Dh, s.Rv * s.Dh};
     L.off[0] = 0;
     for (int i = 0; i < 6; ++i) L.off[i + 1] = L.off[i] + w[i];
     L.dst[0] = f.a_q; L.dst[1] = f.a_k; L.dst[2] = f.a_v;

@@ -97,9 +97,11 @@ def torch_dtype(dtype: str):
 
 
 def factor_widths(n_heads, head_dim, rank_q, rank_k, rank_v):
-    """Rows of the stacked projection weight: W_A_q, W_A_k, W_A_v, W_B_q, W_B_k, W_B_v."""
+    """Rows of the stacked projection weight: W_A_q, W_A_k, W_A_v, W_B_q, W_B_k, W_B_v.
+    TPA-KVonly (rank_q = 0): no W_A_q rows, and the W_B_q block is the plain query
+    projection with n_heads * head_dim rows."""
     return [n_heads * rank_q, n_heads * rank_k, n_heads * rank_v,
-            rank_q * head_dim, rank_k * head_dim, rank_v * head_dim]
+            (rank_q if rank_q > 0 else n_heads) * head_dim, rank_k * head_dim, rank_v * head_dim]
 
 
 # ------------------------------------------------------------------- prefill inputs
@@ -153,17 +155,22 @@ def decode_sequence(wl: Workload, b: int, length: int, a_scale: float = 1.0) -> 
 def prefill_factors(wl: Workload, b: int, n_query: int, n_keys: int, a_scale: float = 1.0) -> dict:
     """Factors for attention-only prefill checks of sequence ``b``: cached K/V factors
     for ``n_keys`` tokens (B_K already rotated) and query factors for ``n_query``
-    tokens (B_Q already rotated), same distributions as ``decode_sequence``."""
+    tokens (B_Q already rotated), same distributions as ``decode_sequence``; for
+    TPA-KVonly the query is ``q`` [n_query, h, d] ~ N(0, 1/d)."""
     h, d, s = wl.n_heads, wl.head_dim, wl.seed
     sd = 1.0 / np.sqrt(d)
-    return {
+    out = {
         "a_k": to_storage(normal(rng(s, "a_k", b), (n_keys, h, wl.rank_k), a_scale), wl.dtype),
         "a_v": to_storage(normal(rng(s, "a_v", b), (n_keys, h, wl.rank_v), a_scale), wl.dtype),
         "b_k": to_storage(normal(rng(s, "b_k", b), (n_keys, wl.rank_k, d), sd), wl.dtype),
         "b_v": to_storage(normal(rng(s, "b_v", b), (n_keys, wl.rank_v, d), sd), wl.dtype),
-        "a_q": to_storage(normal(rng(s, "a_q", b), (n_query, h, wl.rank_q), a_scale), wl.dtype),
-        "b_q": to_storage(normal(rng(s, "b_q", b), (n_query, wl.rank_q, d), sd), wl.dtype),
     }
+    if wl.rank_q == 0:
+        out["q"] = to_storage(normal(rng(s, "q", b), (n_query, h, d), sd), wl.dtype)
+    else:
+        out["a_q"] = to_storage(normal(rng(s, "a_q", b), (n_query, h, wl.rank_q), a_scale), wl.dtype)
+        out["b_q"] = to_storage(normal(rng(s, "b_q", b), (n_query, wl.rank_q, d), sd), wl.dtype)
+    return out
 
 
 def custom(name: str, base: Workload, **changes) -> Workload:

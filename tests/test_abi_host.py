@@ -84,8 +84,14 @@ def test_host_validation_rejects_bad_arguments(bnd):
     # bad dims: odd head_dim, zero rank, factorised-query call with rank_q = 0
     bad = bnd.Dims(64, 4, 15, 2, 1, 1, bnd.F32).c()
     assert _call(bnd, "tpa_cache_append", by(bad), by(c), by(f), 2, 1, sp, None) == 1
+    # TPA-KVonly takes its query from b_q (a_q may be NULL); a missing b_q is invalid
     kvonly = bnd.Dims(64, 4, 16, 0, 1, 1, bnd.F32).c()
-    assert _call(bnd, "tpa_prefill", by(kvonly), by(f), by(c), 2, 1, sp, fake, None) == 2
+    no_q = bnd.tpa_factors(None, None, fake, fake, fake, fake)
+    assert _call(bnd, "tpa_prefill", by(kvonly), by(no_q), by(c), 2, 1, sp, fake, None) == 1
+    assert _call(bnd, "tpa_project", by(kvonly), fake, fake, 2, 4, sp, fake, 8, by(no_q), None) == 1
+    assert _call(bnd, "tpa_prefill", by(kvonly), by(f), by(c), 2, 1, bnd._ints([8, 0]), fake, None) == 3
+    negq = bnd.Dims(64, 4, 16, -1, 1, 1, bnd.F32).c()
+    assert _call(bnd, "tpa_prefill", by(negq), by(f), by(c), 2, 1, sp, fake, None) == 1
     assert _call(bnd, "tpa_rope_table", by(d), 0.5, 8, fake, None) == 1
 
 

@@ -62,9 +62,13 @@ def _project_case(tpa, wl, batch, seqlen, start):
     od = oracle_dims(wl)
     ref = oracle.project(f64(x), f64(w), od)
     pos = np.concatenate([np.arange(s, s + seqlen) for s in start])
+    if wl.rank_q == 0:
+        # TPA-KVonly: the rotated plain query lands in the b_q slot
+        ref["b_q"] = ref.pop("q")
+    names = [n for n in oracle.FACTOR_NAMES if n in ref]
     ref["b_q"] = oracle.rope_rotate(ref["b_q"], pos, wl.rope_base)
     ref["b_k"] = oracle.rope_rotate(ref["b_k"], pos, wl.rope_base)
-    return {n: rel_err(getattr(out, n), ref[n]) for n in oracle.FACTOR_NAMES}
+    return {n: rel_err(getattr(out, n), ref[n]) for n in names}
 
 
 def test_project_tiny_f32(tpa):
@@ -79,6 +83,15 @@ def test_project_bf16_ragged(tpa, wl):
     small = I.custom("proj_small", wl, d_model=256 if wl is C2 else 384)
     errs = _project_case(tpa, small, 3, 173, [0, 5, 1000])
     assert max(errs.values()) < TOL["bf16"], errs
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_project_kvonly(tpa, dtype):
+    """TPA-KVonly: W_Q (h*d_h rows) in the W_B_q slot, rotated per head into b_q."""
+    wl = I.custom("proj_kvonly", C4, dtype=dtype, d_model=256, seed=1011)
+    errs = _project_case(tpa, wl, 2, 150, [0, 700])
+    assert set(errs) == {"b_q", "a_k", "a_v", "b_k", "b_v"}
+    assert max(errs.values()) < TOL[dtype], errs
 
 
 # ------------------------------------------------------------------ cache append
@@ -120,6 +133,11 @@ PREFILL_CASES = [
     (I.custom("p_d128", C5), 2, 150, [0, 90], 1.0),
     (I.custom("p_d128", C5), 1, 1, [300], 8.0),
     (I.custom("p_d128", C5), 1, 256, [0], 8.0),
+    # TPA-KVonly: plain per-head query (rank_q = 0)
+    (I.custom("p_kv_f32", C4, dtype="f32", n_heads=4, head_dim=32), 2, 45, [0, 20], 8.0),
+    (I.custom("p_kv_d128", C4, n_heads=16), 2, 170, [0, 33], 1.0),
+    (I.custom("p_kv_d128", C4, n_heads=16), 1, 150, [64], 8.0),
+    (I.custom("p_kv_d64", C4, n_heads=16, head_dim=64), 2, 131, [7, 0], 8.0),
 ]
 
 
@@ -137,8 +155,11 @@ def test_prefill_from_factors(tpa, case):
         seq = I.prefill_factors(wl, b, S, start[b] + S, a_scale)
         seqs.append(seq)
         fill_cache(cache, b, seq)
-        q.a_q[b * S:(b + 1) * S].copy_(seq["a_q"])
-        q.b_q[b * S:(b + 1) * S].copy_(seq["b_q"])
+        if wl.rank_q == 0:
+            q.b_q[b * S:(b + 1) * S].copy_(seq["q"])     # TPA-KVonly query in the b_q slot
+        else:
+            q.a_q[b * S:(b + 1) * S].copy_(seq["a_q"])
+            q.b_q[b * S:(b + 1) * S].copy_(seq["b_q"])
     out = torch.empty((batch * S, wl.n_heads, wl.head_dim), dtype=dims.torch_dtype, device="cuda")
     tpa.tpa_prefill(dims, q, cache, batch, S, start, out)
     torch.cuda.synchronize()
@@ -235,11 +256,13 @@ E2E_CASES = [
     (TINY, 2, [40, 24]),
     (I.custom("e_d64", C2, d_model=256), 2, [150, 58]),
     (I.custom("e_d128", C5, d_model=256), 2, [130]),
+    (I.custom("e_kv_f32", C4, dtype="f32", d_model=64, n_heads=4, head_dim=16, seed=1012), 2, [33, 20]),
+    (I.custom("e_kv_d128", C4, d_model=256, n_heads=16, seed=1013), 2, [100, 41]),
 ]
 
 
 @pytest.mark.parametrize("case", E2E_CASES,
-                         ids=[f"{c[0].dtype}-d{c[0].head_dim}-chunks{len(c[2])}" for c in E2E_CASES])
+                         ids=[f"{c[0].dtype}-d{c[0].head_dim}-rq{c[0].rank_q}-chunks{len(c[2])}" for c in E2E_CASES])
 def test_layer_prefill_end_to_end(tpa, case):
     """project -> append -> prefill from x, in one or two chunks (second chunk at
     start_pos > 0), against the pages' forward evaluated in fp64."""
