@@ -56,13 +56,19 @@ PROFILED_TRAFFIC = {
 def attn_flops_per_pair(wl) -> int:
     """Algorithmic flops per (query, key) pair, all heads: the B-space score
     contraction 2 R_Q R_K d_h, its per-head a_Q a_K weighting 2 h R_Q R_K, and the
-    weighted sum of values 2 h d_h."""
+    weighted sum of values 2 h d_h.  TPA-KVonly: the per-head query against each
+    B_K row, 2 h R_K d_h, the a_K weighting 2 h R_K, and the values 2 h d_h."""
+    if wl.rank_q == 0:
+        return 2 * wl.n_heads * wl.rank_k * wl.head_dim + 2 * wl.n_heads * wl.rank_k \
+            + 2 * wl.n_heads * wl.head_dim
     return 2 * wl.rank_q * wl.rank_k * wl.head_dim + 2 * wl.n_heads * wl.rank_q * wl.rank_k \
         + 2 * wl.n_heads * wl.head_dim
 
 
 def proj_flops(wl, tokens: int) -> int:
     n = (wl.rank_q + wl.rank_k + wl.rank_v) * (wl.n_heads + wl.head_dim)
+    if wl.rank_q == 0:
+        n += wl.n_heads * wl.head_dim              # TPA-KVonly: the plain W_Q
     return 2 * tokens * n * wl.d_model
 
 
@@ -446,10 +452,13 @@ def oracle_decode_sample(wl, n_seq: int = 1, length: int | None = None):
 
 def cpu_baseline(wl):
     if wl.kind == "prefill":
-        dt, fl = oracle_prefill_sample(wl, 1)
+        # a bounded sample: at most 2048 tokens of one sequence (the fp64 scores alone
+        # are h * S^2 * 8 bytes)
+        S = min(wl.seqlen, 2048)
+        dt, fl = oracle_prefill_sample(wl, 1, seqlen=S)
         return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
-                "sample": f"fp64 oracle forward of 1 of {wl.batch} sequences ({wl.seqlen} tokens): "
-                          f"projection, RoPE, causal attention; {dt:.1f} s"}
+                "sample": f"fp64 oracle forward of the first {S} tokens of 1 of {wl.batch} sequences "
+                          f"({wl.seqlen} tokens each): projection, RoPE, causal attention; {dt:.1f} s"}
     dt, by = oracle_decode_sample(wl, 2)
     return {"value": by / dt / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
             "sample": f"fp64 oracle decode of 2 of {wl.batch} sequences; {dt:.1f} s"}

@@ -67,6 +67,11 @@ WORKLOADS = {
         Workload("layer_prefill_b4_s8192_d2048", "prefill", "bf16", batch=4, seqlen=8192,
                  d_model=2048, n_heads=16, head_dim=128, rank_q=6, rank_k=2, rank_v=2,
                  rope_base=1e4, seed=1005),
+        # TPA-KVonly layer prefill: the KV-only decode shape (h 32, d_h 128, R 2, base
+        # 5e5) with d_model = h * d_h; a measurement case for the KV-only prefill path
+        Workload("kvonly_layer_prefill_b4_s8192_d4096", "prefill", "bf16", batch=4, seqlen=8192,
+                 d_model=4096, n_heads=32, head_dim=128, rank_q=0, rank_k=2, rank_v=2,
+                 rope_base=5e5, seed=1006),
     )
 }
 

@@ -52,6 +52,11 @@ def test_full_layer_prefill_b4_s8192_d2048(tpa):
     _full_prefill(tpa, wl, [wl.batch - 1], _rows(wl.seqlen, 40, 2))
 
 
+def test_full_kvonly_layer_prefill_b4_s8192_d4096(tpa):
+    wl = I.WORKLOADS["kvonly_layer_prefill_b4_s8192_d4096"]
+    _full_prefill(tpa, wl, [wl.batch - 1], _rows(wl.seqlen, 24, 3))
+
+
 def _full_decode(tpa, wl, sample):
     dims = dims_of(wl, tpa)
     lengths = [int(v) for v in I.decode_lengths(wl)]
