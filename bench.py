@@ -236,16 +236,15 @@ class PrefillStep:
         self.xn = self.xn_host.cuda()
         self.w = I.prefill_w(wl).cuda()
         self.fac = tpa.alloc_factors(self.dims, B * S)
-        self.fac1 = tpa.alloc_factors(self.dims, B)
         self.cache = tpa.alloc_cache(self.dims, B, self.cap)
         tdt = self.dims.torch_dtype
         self.out = torch.empty((B * S, wl.n_heads, wl.head_dim), dtype=tdt, device="cuda")
         self.out1 = torch.empty((B, wl.n_heads, wl.head_dim), dtype=tdt, device="cuda")
-        self.lengths = [S + 1] * B
-        self.ws = tpa.alloc_workspace(self.dims, self.lengths)
+        self.pre = [S] * B                     # lengths before the decode step
+        self.ws = tpa.alloc_step_workspace(self.dims, self.pre)
         self.out_host = torch.empty(self.out.shape, dtype=tdt).pin_memory()
         self.out1_host = torch.empty(self.out1.shape, dtype=tdt).pin_memory()
-        self.launches_per_step = 7   # project, append, prefill, project, append, decode, combine
+        self.launches_per_step = 6   # project, append, prefill; decode step: project, decode, combine
 
     def flops(self):
         wl = self.wl
@@ -264,10 +263,7 @@ class PrefillStep:
         mark("append"); t.tpa_cache_append(d, self.cache, self.fac, B, S, zero); done("append")
         mark("prefill"); t.tpa_prefill(d, self.fac, self.cache, B, S, zero, self.out); done("prefill")
         mark("decode_step")
-        pos = [S] * B
-        t.tpa_project(d, self.xn, self.w, B, 1, pos, self.cs, self.cap, self.fac1)
-        t.tpa_cache_append(d, self.cache, self.fac1, B, 1, pos)
-        t.tpa_decode(d, self.fac1.a_q, self.fac1.b_q, self.cache, self.lengths, self.out1, self.ws)
+        t.tpa_decode_step(d, self.xn, self.w, self.cs, self.cap, self.cache, self.pre, self.out1, self.ws)
         done("decode_step")
 
     def run_e2e(self):

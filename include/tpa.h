@@ -186,6 +186,34 @@ tpa_status tpa_decode(const tpa_dims* dims, const void* q_a, const void* q_b,
 /* Workspace bytes tpa_decode needs for these lengths (0 for invalid arguments). */
 size_t tpa_decode_workspace_bytes(const tpa_dims* dims, const int32_t* lengths, int32_t batch);
 
+/* One decode step from the hidden state of the new token of every sequence: project
+ * it (the six projections with RoPE at position lengths[b], as tpa_project), write
+ * its A_K, A_V, B_K, B_V into the cache at position lengths[b] and set
+ * cache->lengths[b] = lengths[b] + 1 (as tpa_cache_append), then decode its query
+ * over keys 0..lengths[b] (as tpa_decode).  This is the page's forward for one token
+ * with start_pos = lengths[b]: project, write the cache, read it back, attend
+ * [review, 代码 前向传播].  Two stream-ordered kernel launches plus decode's merge:
+ * the projection's epilogue writes the key/value factors straight into the cache,
+ * so they never pass through a separate buffer.
+ *   x        device [batch][d_model]: the new token of each sequence
+ *   w_cat    device stacked weights, as tpa_project (TPA-KVonly layout at rank_q = 0)
+ *   rope_cs  device table from tpa_rope_table with max_pos rows; lengths[b] < max_pos
+ *   cache    holds positions 0 .. lengths[b]-1 of sequence b; lengths[b] + 1 <= capacity
+ *   lengths  host [batch], lengths[b] >= 0: the cached length before this step
+ *   out      device [batch][h][d_h]
+ *   workspace device scratch of at least tpa_decode_step_workspace_bytes() bytes,
+ *            256-byte aligned: the new tokens' query factors, then decode's partials.
+ * Arguments are checked before anything is launched (TPA_ERR_CAPACITY when a
+ * sequence has no room or its position is past the RoPE table). */
+tpa_status tpa_decode_step(const tpa_dims* dims, const void* x, const void* w_cat,
+                           const float* rope_cs, int32_t max_pos, const tpa_cache* cache,
+                           const int32_t* lengths, int32_t batch, void* out,
+                           void* workspace, size_t workspace_bytes, tpa_stream_t stream);
+
+/* Workspace bytes tpa_decode_step needs for these pre-step lengths (0 if invalid). */
+size_t tpa_decode_step_workspace_bytes(const tpa_dims* dims, const int32_t* lengths,
+                                       int32_t batch);
+
 /* tpa_decode without a caller-supplied workspace, for callers that cannot allocate
  * device memory: a host application that owns every allocation and hands this
  * library only its inputs and outputs, or a server that must not call cudaMalloc

@@ -27,8 +27,8 @@ TPA_MAX_BATCH = 1024
 # Every symbol include/tpa.h declares (checked by tests/test_abi_host.py).
 EXPORTS = ("tpa_abi_version", "tpa_build_info", "tpa_status_string", "tpa_cache_bytes_per_token",
            "tpa_rope_table", "tpa_project", "tpa_cache_append", "tpa_prefill", "tpa_decode",
-           "tpa_decode_workspace_bytes", "tpa_decode_static", "tpa_get_device_error",
-           "tpa_set_wait_limit")
+           "tpa_decode_workspace_bytes", "tpa_decode_static", "tpa_decode_step",
+           "tpa_decode_step_workspace_bytes", "tpa_get_device_error", "tpa_set_wait_limit")
 TPA_DECODE_STATIC_SCRATCH_BYTES = 16 << 20
 
 
@@ -70,6 +70,10 @@ _sig = {
     "tpa_decode_workspace_bytes": (ctypes.c_size_t, [_P(tpa_dims), _i32p, ctypes.c_int32]),
     "tpa_decode_static": (ctypes.c_int, [_P(tpa_dims), ctypes.c_void_p, ctypes.c_void_p, _P(tpa_cache),
                                          _i32p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]),
+    "tpa_decode_step": (ctypes.c_int, [_P(tpa_dims), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_int32, _P(tpa_cache), _i32p, ctypes.c_int32,
+                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "tpa_decode_step_workspace_bytes": (ctypes.c_size_t, [_P(tpa_dims), _i32p, ctypes.c_int32]),
     "tpa_get_device_error": (ctypes.c_int, [ctypes.c_void_p, _i32p]),
     "tpa_set_wait_limit": (None, [ctypes.c_uint32]),
 }
@@ -257,6 +261,29 @@ def tpa_decode_static(dims: Dims, q_a, q_b, cache: Cache, lengths, out, stream=N
     _check("tpa_decode_static", _lib.tpa_decode_static(ctypes.byref(dims.c()), _ptr(q_a), _ptr(q_b),
                                                        ctypes.byref(cache.c()), _ints(lengths), len(lengths),
                                                        _ptr(out), _stream(stream)))
+
+
+def tpa_decode_step_workspace_bytes(dims: Dims, lengths) -> int:
+    lengths = list(lengths)
+    return _lib.tpa_decode_step_workspace_bytes(ctypes.byref(dims.c()), _ints(lengths), len(lengths))
+
+
+def tpa_decode_step(dims: Dims, x, w_cat, rope_cs, max_pos: int, cache: Cache, lengths, out,
+                    workspace, stream=None) -> None:
+    """Project the new token of every sequence, append its K/V factors at lengths[b]
+    (advancing cache.lengths) and decode it; ``lengths`` are the pre-step lengths."""
+    lengths = list(lengths)
+    _check("tpa_decode_step", _lib.tpa_decode_step(
+        ctypes.byref(dims.c()), _ptr(x), _ptr(w_cat), _ptr(rope_cs), int(max_pos),
+        ctypes.byref(cache.c()), _ints(lengths), len(lengths), _ptr(out), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def alloc_step_workspace(dims: Dims, lengths, device="cuda") -> torch.Tensor:
+    n = tpa_decode_step_workspace_bytes(dims, lengths)
+    if n == 0:
+        raise ValueError("invalid decode-step arguments")
+    return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def tpa_get_device_error(stream=None) -> int:

@@ -29,10 +29,10 @@ __device__ __forceinline__ int segment_of(const ProjLayout& L, int c) {
 }
 
 template <typename T>
-__device__ __forceinline__ void store_col(const ProjLayout& L, int seg, int t, int c, float v) {
+__device__ __forceinline__ void store_col(const ProjLayout& L, int seg, int t, long long tkv, int c, float v) {
     int width = L.off[seg + 1] - L.off[seg];
     T* dst = reinterpret_cast<T*>(L.dst[seg]);
-    dst[(long long)t * width + (c - L.off[seg])] = from_f<T>(v);
+    dst[seg_row(L, seg, t, tkv) * width + (c - L.off[seg])] = from_f<T>(v);
 }
 
 template <typename T>
@@ -76,6 +76,9 @@ __global__ void __launch_bounds__(NT) project_simt_kernel(ProjArgs a, SeqParams 
         if (t >= a.T) continue;
         int b = t / a.seqlen;
         int pos = start.v[b] + (t - b * a.seqlen);
+        const long long tkv = (long long)b * L.kv_cap + pos;
+        // cache mode: the sequence's last token records the new length, once
+        if (L.lengths && col0 == 0 && tx == 0 && t - b * a.seqlen == a.seqlen - 1) L.lengths[b] = pos + 1;
 #pragma unroll
         for (int jp = 0; jp < 2; ++jp) {
             int c = col0 + tx * 4 + 2 * jp;
@@ -87,11 +90,11 @@ __global__ void __launch_bounds__(NT) project_simt_kernel(ProjArgs a, SeqParams 
                 int local = c - L.off[seg];
                 int k2 = (local % a.Dh) >> 1;
                 float2 r = a.cs[(long long)pos * (a.Dh >> 1) + k2];
-                store_col<T>(L, seg, t, c, y0 * r.x - y1 * r.y);
-                store_col<T>(L, seg, t, c + 1, y0 * r.y + y1 * r.x);
+                store_col<T>(L, seg, t, tkv, c, y0 * r.x - y1 * r.y);
+                store_col<T>(L, seg, t, tkv, c + 1, y0 * r.y + y1 * r.x);
             } else {
-                store_col<T>(L, seg, t, c, y0);
-                if (c + 1 < a.N) store_col<T>(L, segment_of(L, c + 1), t, c + 1, y1);
+                store_col<T>(L, seg, t, tkv, c, y0);
+                if (c + 1 < a.N) store_col<T>(L, segment_of(L, c + 1), t, tkv, c + 1, y1);
             }
         }
     }

@@ -44,14 +44,15 @@ __device__ __forceinline__ int seg_of(const ProjLayout& L, int c) {
     return s;
 }
 
-// Store output columns [c0, min(c0+16, N)) of token t (v already rotated).
-__device__ __forceinline__ void store16(const ProjLayout& L, int N, long long t, int c0,
+// Store output columns [c0, min(c0+16, N)) of token t (v already rotated); tkv is the
+// token's cache row (cache mode).
+__device__ __forceinline__ void store16(const ProjLayout& L, int N, long long t, long long tkv, int c0,
                                         const float (&v)[16]) {
     const int s0 = seg_of(L, c0);
     const int last = min(c0 + 15, N - 1);
     if (c0 + 15 < N && seg_of(L, last) == s0) {
         const int width = L.off[s0 + 1] - L.off[s0];
-        const long long e = t * width + (c0 - L.off[s0]);
+        const long long e = seg_row(L, s0, t, tkv) * width + (c0 - L.off[s0]);
         __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(L.dst[s0]) + e;
         if ((e & 7) == 0) {
             uint4 w0, w1;
@@ -70,7 +71,7 @@ __device__ __forceinline__ void store16(const ProjLayout& L, int N, long long t,
         if (c < N) {
             const int s = seg_of(L, c);
             const int width = L.off[s + 1] - L.off[s];
-            reinterpret_cast<__nv_bfloat16*>(L.dst[s])[t * width + (c - L.off[s])] =
+            reinterpret_cast<__nv_bfloat16*>(L.dst[s])[seg_row(L, s, t, tkv) * width + (c - L.off[s])] =
                 __float2bfloat16_rn(v[j]);
         }
     }
@@ -187,9 +188,14 @@ project_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
             const long long t = (long long)m * BM + row;
             const bool valid = t < a.T;
             int pos = 0;
+            long long tkv = 0;
             if (valid) {
                 const int b = (int)(t / a.seqlen);
-                pos = start.v[b] + (int)(t - (long long)b * a.seqlen);
+                const int i = (int)(t - (long long)b * a.seqlen);
+                pos = start.v[b] + i;
+                tkv = (long long)b * a.L.kv_cap + pos;
+                // cache mode: the sequence's last token records the new length, once
+                if (a.L.lengths && n == 0 && colhalf == 0 && i == a.seqlen - 1) a.L.lengths[b] = pos + 1;
             }
             const int col0 = n * a.BN;
             const int cend = min(a.N, col0 + a.BN);
@@ -218,8 +224,8 @@ project_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
                     v[2 * j] = x0 * rot[j].x - x1 * rot[j].y;
                     v[2 * j + 1] = x0 * rot[j].y + x1 * rot[j].x;
                 }
-                store16(a.L, cend, t, cg, *reinterpret_cast<float(*)[16]>(&v[0]));
-                if (cg + 16 < cend) store16(a.L, cend, t, cg + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+                store16(a.L, cend, t, tkv, cg, *reinterpret_cast<float(*)[16]>(&v[0]));
+                if (cg + 16 < cend) store16(a.L, cend, t, tkv, cg + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
             }
             tc_fence_before();
             __syncwarp();

@@ -67,6 +67,42 @@ tpa_status check_cache(const tpa_cache* c, int batch) {
 
 tpa_status launched(cudaError_t e) { return e == cudaSuccess ? TPA_OK : TPA_ERR_CUDA; }
 
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Workspace bytes tpa_decode_step keeps for the new tokens' query factors (a_q, then
+// b_q or the KV-only query), each 256-byte aligned.
+size_t step_query_bytes(const Shape& s, int batch) {
+    const size_t es = s.bf16 ? 2 : 4;
+    const size_t q_rows = s.Rq > 0 ? (size_t)s.Rq : (size_t)s.H;
+    return round_up((size_t)batch * s.H * s.Rq * es, 256) + round_up((size_t)batch * q_rows * s.Dh * es, 256);
+}
+
+// The projection GEMM with its fused epilogue (validated arguments).
+tpa_status run_project(const Shape& s, const void* x, const void* w, int batch, int seqlen,
+                       const SeqParams& sp, const float* rope_cs, const ProjLayout& L,
+                       cudaStream_t cs) {
+    if (s.bf16 && project_tc_supported(s, batch * seqlen))
+        return launched(launch_project_tc(s, x, w, batch, seqlen, sp, rope_cs, L,
+                                          device_error_ptr(), wait_limit(), cs));
+    return launched(launch_project_simt(s, x, w, batch, seqlen, sp, rope_cs, L, cs));
+}
+
+// Split-K decode and the fixed-order merge of its parts (validated arguments).
+tpa_status run_decode(const Shape& s, const void* q_a, const void* q_b, const tpa_cache& c,
+                      const int32_t* lengths, int batch, void* out, void* workspace,
+                      size_t workspace_bytes, cudaStream_t cs) {
+    const bool tc = s.bf16 && decode_tc_supported(s);
+    if (!tc && (long long)s.H * s.Dh > 8192) return TPA_ERR_UNSUPPORTED;
+    DecodePlan plan;
+    make_decode_plan(s, lengths, batch, tc, &plan);
+    if (decode_workspace_bytes(s, plan) > workspace_bytes) return TPA_ERR_WORKSPACE;
+    float* ws = static_cast<float*>(workspace);
+    cudaError_t e = tc ? launch_decode_tc(s, q_a, q_b, c, plan, ws, device_error_ptr(), wait_limit(), cs)
+                       : launch_decode_simt(s, q_a, q_b, c, plan, ws, cs);
+    if (e != cudaSuccess) return TPA_ERR_CUDA;
+    return launched(launch_decode_combine(s, plan, ws, out, cs));
+}
+
 }  // namespace
 
 extern "C" {
@@ -130,12 +166,8 @@ tpa_status tpa_project(const tpa_dims* d, const void* x, const void* w_cat, int3
         sp.v[b] = start_pos[b];
     }
     Shape s = shape_of(*d);
-    ProjLayout L = proj_layout(s, *out);
-    cudaStream_t cs = (cudaStream_t)stream;
-    if (s.bf16 && project_tc_supported(s, batch * seqlen))
-        return launched(launch_project_tc(s, x, w_cat, batch, seqlen, sp, rope_cs, L,
-                                          device_error_ptr(), wait_limit(), cs));
-    return launched(launch_project_simt(s, x, w_cat, batch, seqlen, sp, rope_cs, L, cs));
+    return run_project(s, x, w_cat, batch, seqlen, sp, rope_cs, proj_layout(s, *out),
+                       (cudaStream_t)stream);
 }
 
 tpa_status tpa_cache_append(const tpa_dims* d, const tpa_cache* c, const tpa_factors* kv,
@@ -210,19 +242,72 @@ tpa_status tpa_decode(const tpa_dims* d, const void* q_a, const void* q_b,
         if (lengths[b] < 1) return TPA_ERR_INVALID;
         if (lengths[b] > c->capacity) return TPA_ERR_CAPACITY;
     }
+    return run_decode(shape_of(*d), q_a, q_b, *c, lengths, batch, out, workspace, workspace_bytes,
+                      (cudaStream_t)stream);
+}
+
+size_t tpa_decode_step_workspace_bytes(const tpa_dims* d, const int32_t* lengths, int32_t batch) {
+    if (check_dims(d, false) != TPA_OK || !lengths || batch < 1 || batch > TPA_MAX_BATCH)
+        return 0;
+    int32_t next[TPA_MAX_BATCH];
+    for (int b = 0; b < batch; ++b) {
+        if (lengths[b] < 0) return 0;
+        next[b] = lengths[b] + 1;
+    }
     Shape s = shape_of(*d);
-    const bool tc = s.bf16 && decode_tc_supported(s);
-    if (!tc && (long long)s.H * s.Dh > 8192) return TPA_ERR_UNSUPPORTED;
     DecodePlan plan;
-    make_decode_plan(s, lengths, batch, tc, &plan);
-    if (decode_workspace_bytes(s, plan) > workspace_bytes) return TPA_ERR_WORKSPACE;
+    make_decode_plan(s, next, batch, s.bf16 && decode_tc_supported(s), &plan);
+    return step_query_bytes(s, batch) + decode_workspace_bytes(s, plan);
+}
+
+tpa_status tpa_decode_step(const tpa_dims* d, const void* x, const void* w_cat,
+                           const float* rope_cs, int32_t max_pos, const tpa_cache* c,
+                           const int32_t* lengths, int32_t batch, void* out,
+                           void* workspace, size_t workspace_bytes, tpa_stream_t stream) {
+    tpa_status st = check_dims(d, false);
+    if (st != TPA_OK) return st;
+    if ((st = check_cache(c, batch)) != TPA_OK) return st;
+    if (d->d_model < 1) return TPA_ERR_INVALID;
+    if (!x || !w_cat || !rope_cs || !lengths || !out || !workspace) return TPA_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(w_cat) || !aligned16(rope_cs) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return TPA_ERR_INVALID;
+    if ((d->n_heads * (d->rank_q + d->rank_k + d->rank_v)) & 1) return TPA_ERR_UNSUPPORTED;
+    SeqParams sp;
+    int32_t next[TPA_MAX_BATCH];
+    for (int b = 0; b < batch; ++b) {
+        if (lengths[b] < 0 || max_pos < 1) return TPA_ERR_INVALID;
+        if (lengths[b] >= max_pos || lengths[b] + 1 > c->capacity) return TPA_ERR_CAPACITY;
+        sp.v[b] = lengths[b];
+        next[b] = lengths[b] + 1;
+    }
+    Shape s = shape_of(*d);
+    const size_t qb = step_query_bytes(s, batch);
+    if (workspace_bytes < qb) return TPA_ERR_WORKSPACE;
+    // the new token's query factors go to the front of the workspace; its K/V factors
+    // go straight into the cache rows lengths[b], and cache->lengths[b] is advanced
+    const size_t es = s.bf16 ? 2 : 4;
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    const size_t aq_bytes = round_up((size_t)batch * s.H * s.Rq * es, 256);
+    tpa_factors f;
+    f.a_q = s.Rq > 0 ? wsb : nullptr;
+    f.b_q = wsb + aq_bytes;
+    f.a_k = c->a_k; f.a_v = c->a_v; f.b_k = c->b_k; f.b_v = c->b_v;
+    ProjLayout L = proj_layout(s, f);
+    L.kv_cap = c->capacity;
+    L.lengths = c->lengths;
     cudaStream_t cs = (cudaStream_t)stream;
-    float* ws = static_cast<float*>(workspace);
-    cudaError_t e = tc ? launch_decode_tc(s, q_a, q_b, *c, plan, ws, device_error_ptr(),
-                                          wait_limit(), cs)
-                       : launch_decode_simt(s, q_a, q_b, *c, plan, ws, cs);
-    if (e != cudaSuccess) return TPA_ERR_CUDA;
-    return launched(launch_decode_combine(s, plan, ws, out, cs));
+    // check the decode half before anything is launched
+    {
+        const bool tc = s.bf16 && decode_tc_supported(s);
+        if (!tc && (long long)s.H * s.Dh > 8192) return TPA_ERR_UNSUPPORTED;
+        DecodePlan plan;
+        make_decode_plan(s, next, batch, tc, &plan);
+        if (qb + decode_workspace_bytes(s, plan) > workspace_bytes) return TPA_ERR_WORKSPACE;
+    }
+    st = run_project(s, x, w_cat, batch, 1, sp, rope_cs, L, cs);
+    if (st != TPA_OK) return st;
+    return run_decode(s, f.a_q, f.b_q, *c, next, batch, out, wsb + qb, workspace_bytes - qb, cs);
 }
 
 tpa_status tpa_get_device_error(tpa_stream_t stream, int32_t* code) {

@@ -31,7 +31,17 @@ inline Shape shape_of(const tpa_dims& d) {
 struct ProjLayout {
     int off[7];    // segment starts, off[6] = N
     void* dst[6];  // a_q, a_k, a_v, b_q, b_k, b_v
+    // Cache mode (kv_cap > 0): dst[1,2,4,5] are the cache's a_k, a_v, b_k, b_v and
+    // token t = b*seqlen + i lands in cache row b*kv_cap + start[b] + i; the kernel
+    // also sets lengths[b] = start[b] + seqlen.  Otherwise every segment is at row t.
+    int kv_cap = 0;
+    int32_t* lengths = nullptr;
 };
+
+// Destination row of segment s for token t (tkv: its cache row in cache mode).
+__host__ __device__ inline long long seg_row(const ProjLayout& L, int s, long long t, long long tkv) {
+    return (L.kv_cap > 0 && s != 0 && s != 3) ? tkv : t;
+}
 
 inline ProjLayout proj_layout(const Shape& s, const tpa_factors& f) {
     ProjLayout L;

@@ -95,6 +95,28 @@ def test_host_validation_rejects_bad_arguments(bnd):
     assert _call(bnd, "tpa_rope_table", by(d), 0.5, 8, fake, None) == 1
 
 
+def test_decode_step_host_validation(bnd):
+    d = bnd.Dims(64, 4, 16, 2, 1, 1, bnd.F32).c()
+    by = ctypes.byref
+    fake = 0x10000
+    c = bnd.tpa_cache(fake, fake, fake, fake, fake, 2, 8)
+    need = bnd.tpa_decode_step_workspace_bytes(bnd.Dims(64, 4, 16, 2, 1, 1, bnd.F32), [3, 5])
+    assert need > bnd.tpa_decode_workspace_bytes(bnd.Dims(64, 4, 16, 2, 1, 1, bnd.F32), [4, 6])
+    step = lambda *a: _call(bnd, "tpa_decode_step", *a)
+    ok = (fake, fake, fake, 16, by(c), bnd._ints([3, 5]), 2, fake, fake, need, None)
+    # null input, misaligned workspace, workspace too small
+    assert step(by(d), None, *ok[1:]) == 1
+    assert step(by(d), *ok[:8], fake + 16, need, None) == 1
+    assert step(by(d), *ok[:9], need - 4, None) == 5
+    # no room in the cache (capacity 8), position past the RoPE table (max_pos 6)
+    assert step(by(d), fake, fake, fake, 16, by(c), bnd._ints([3, 8]), 2, fake, fake, need, None) == 3
+    assert step(by(d), fake, fake, fake, 6, by(c), bnd._ints([3, 6]), 2, fake, fake, need, None) == 3
+    # negative length, batch larger than the cache
+    assert step(by(d), fake, fake, fake, 16, by(c), bnd._ints([-1, 5]), 2, fake, fake, need, None) == 1
+    assert step(by(d), fake, fake, fake, 16, by(c), bnd._ints([1, 1, 1]), 3, fake, fake, need, None) == 1
+    assert bnd.tpa_decode_step_workspace_bytes(bnd.Dims(64, 4, 16, 2, 1, 1, bnd.F32), [-1]) == 0
+
+
 def test_workspace_size_formula(bnd):
     dims = bnd.Dims(0, 16, 128, 6, 2, 2)
     lengths = [32768] * 64

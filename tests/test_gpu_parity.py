@@ -310,3 +310,58 @@ def test_decode_step_after_prefill_end_to_end(tpa):
     torch.cuda.synchronize()
     ref, _ = oracle.tpa_forward(np.stack([f64(xb) for xb in xs]), f64(w), oracle_dims(wl), wl.rope_base)
     assert rel_err(out, ref[:, S]) < TOL["bf16"]
+
+
+# ------------------------------------------------------------ fused decode step
+
+STEP_CASES = [
+    # (workload, pre-step lengths)
+    (I.custom("s_d128", C5, d_model=256), [97, 40, 1]),
+    (I.custom("s_kv", C4, d_model=256, n_heads=16, seed=1014), [64, 133]),
+    (I.custom("s_f32", TINY), [30, 0]),
+]
+
+
+@pytest.mark.parametrize("case", STEP_CASES,
+                         ids=[f"{c[0].dtype}-d{c[0].head_dim}-rq{c[0].rank_q}" for c in STEP_CASES])
+def test_decode_step_fused(tpa, case):
+    """tpa_decode_step (project the new token straight into the cache, then decode)
+    against the pages' forward over lengths[b] + 1 tokens, and against the separate
+    project -> append path for the cache rows it writes (bit for bit)."""
+    wl, lengths = case
+    dims = dims_of(wl, tpa)
+    B, cap = len(lengths), max(lengths) + 3
+    max_pos = cap
+    cs = rope_table(tpa, dims, wl.rope_base, max_pos)
+    xs = [I.prefill_x(wl, b, L + 1) for b, L in enumerate(lengths)]
+    w = I.prefill_w(wl)
+    wd = w.cuda()
+    cache = tpa.alloc_cache(dims, B, cap, fill=float("nan"))
+    twin = tpa.alloc_cache(dims, B, cap, fill=float("nan"))
+    for b, L in enumerate(lengths):
+        if L == 0:
+            continue
+        fac = tpa.alloc_factors(dims, L)
+        tpa.tpa_project(dims, xs[b][:L].cuda(), wd, 1, L, [0], cs, max_pos, fac)
+        one = tpa.Cache(*(getattr(cache, n)[b:b + 1] for n in ("a_k", "a_v", "b_k", "b_v")), cache.lengths[b:b + 1])
+        tpa.tpa_cache_append(dims, one, fac, 1, L, [0])
+        for n in ("a_k", "a_v", "b_k", "b_v"):
+            getattr(twin, n)[b].copy_(getattr(cache, n)[b])
+    xn = torch.stack([xs[b][L] for b, L in enumerate(lengths)]).cuda()
+    out = torch.empty((B, wl.n_heads, wl.head_dim), dtype=dims.torch_dtype, device="cuda")
+    tpa.tpa_decode_step(dims, xn, wd, cs, max_pos, cache, lengths, out, tpa.alloc_step_workspace(dims, lengths))
+    # the same token through the separate calls, into the twin cache
+    fac1 = tpa.alloc_factors(dims, B)
+    tpa.tpa_project(dims, xn, wd, B, 1, lengths, cs, max_pos, fac1)
+    tpa.tpa_cache_append(dims, twin, fac1, B, 1, lengths)
+    torch.cuda.synchronize()
+    assert tpa.tpa_get_device_error() == 0
+    assert cache.lengths.cpu().tolist() == [L + 1 for L in lengths]
+    ibits = torch.int16 if wl.dtype == "bf16" else torch.int32
+    for n in ("a_k", "a_v", "b_k", "b_v"):
+        for b, L in enumerate(lengths):
+            assert torch.equal(getattr(cache, n)[b, L].view(ibits), getattr(twin, n)[b, L].view(ibits)), (n, b)
+    od = oracle_dims(wl)
+    for b, L in enumerate(lengths):
+        ref = oracle.tpa_forward_rows(f64(xs[b]), f64(w), od, wl.rope_base, [L])
+        assert rel_err(out[b:b + 1], ref) < TOL[wl.dtype], b
