@@ -302,6 +302,17 @@ def decode_attention(q_factors: dict, kv: dict, dims: Dims, length: int,
     return out
 
 
+def output_projection(out: np.ndarray, w_o: np.ndarray) -> np.ndarray:
+    """The layer's closing ``self.wo(output)`` ([review] 前向传播): the attention output
+    [T, h, d] is flattened per token to h*d features (``transpose(1,2).view(bsz,
+    seqlen, -1)``) and mapped to d_model by a bias-free linear map.  The page uses
+    ``wo`` without defining it; reading taken: nn.Linear(h*d, d_model, bias=False),
+    w_o of shape [d_model, h*d].  The T6GroupNorm the page constructs is not applied
+    in its forward and is left out."""
+    o = np.asarray(out, dtype=np.float64)
+    return o.reshape(o.shape[0], -1) @ np.asarray(w_o, dtype=np.float64).T
+
+
 def tpa_forward_rows(x: np.ndarray, w_cat: np.ndarray, dims: Dims, rope_base: float,
                      rows) -> np.ndarray:
     """``tpa_forward`` for one sequence that starts at position 0, evaluated only for

@@ -463,3 +463,16 @@ def test_kvonly_forward_is_textbook_attention_on_rotated_q_and_materialised_kv()
         assert rel(oracle.attend_from_factors(qf, kv, dims, np.arange(S)), out[b]) < 1e-12
     rows = [0, 6, 10]
     assert rel(oracle.tpa_forward_rows(x[1], w_cat, dims, base, rows), out[1, rows]) < 1e-12
+
+
+def test_output_projection_is_a_bias_free_linear_on_flattened_heads():
+    # [review] 前向传播: output.transpose(1, 2).contiguous().view(bsz, seqlen, -1), then wo
+    g = gen(23)
+    T, h, d, D = 6, 3, 4, 10
+    out = g.standard_normal((T, h, d))
+    w_o = g.standard_normal((D, h * d))
+    want = F.linear(torch.from_numpy(out).reshape(T, h * d), torch.from_numpy(w_o)).numpy()
+    assert rel(oracle.output_projection(out, w_o), want) < TOL
+    # head-major flattening: feature h*d + k of the input is head h, dim k
+    e = np.zeros((1, h, d)); e[0, 2, 1] = 1.0
+    assert rel(oracle.output_projection(e, w_o)[0], w_o[:, 2 * d + 1]) < TOL
