@@ -210,6 +210,18 @@ tpa_status tpa_decode_step(const tpa_dims* dims, const void* x, const void* w_ca
                            const int32_t* lengths, int32_t batch, void* out,
                            void* workspace, size_t workspace_bytes, tpa_stream_t stream);
 
+/* Output projection: out = attn W_o^T, the layer's closing self.wo(output) [review, 代码
+ * 前向传播], with the attention output flattened head-major per token (feature
+ * h*d_h + k is head h, dim k, as transpose(1,2).view(bsz, seqlen, -1)).  The page
+ * uses wo without defining it; reading taken: a bias-free nn.Linear(h*d_h, d_model).
+ * The T6GroupNorm the page constructs is not applied in its forward and is not here.
+ *   attn  device [T][h][d_h] (tpa_prefill's or tpa_decode's out)
+ *   w_o   device [d_model][h*d_h]
+ *   out   device [T][d_model]
+ * Same element type throughout (dims->dtype); fp32 accumulation. */
+tpa_status tpa_output_project(const tpa_dims* dims, const void* attn, const void* w_o,
+                              int32_t T, void* out, tpa_stream_t stream);
+
 /* Workspace bytes tpa_decode_step needs for these pre-step lengths (0 if invalid). */
 size_t tpa_decode_step_workspace_bytes(const tpa_dims* dims, const int32_t* lengths,
                                        int32_t batch);

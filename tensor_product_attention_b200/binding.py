@@ -28,7 +28,8 @@ TPA_MAX_BATCH = 1024
 EXPORTS = ("tpa_abi_version", "tpa_build_info", "tpa_status_string", "tpa_cache_bytes_per_token",
            "tpa_rope_table", "tpa_project", "tpa_cache_append", "tpa_prefill", "tpa_decode",
            "tpa_decode_workspace_bytes", "tpa_decode_static", "tpa_decode_step",
-           "tpa_decode_step_workspace_bytes", "tpa_get_device_error", "tpa_set_wait_limit")
+           "tpa_decode_step_workspace_bytes", "tpa_output_project", "tpa_get_device_error",
+           "tpa_set_wait_limit")
 TPA_DECODE_STATIC_SCRATCH_BYTES = 16 << 20
 
 
@@ -74,6 +75,8 @@ _sig = {
                                        ctypes.c_int32, _P(tpa_cache), _i32p, ctypes.c_int32,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "tpa_decode_step_workspace_bytes": (ctypes.c_size_t, [_P(tpa_dims), _i32p, ctypes.c_int32]),
+    "tpa_output_project": (ctypes.c_int, [_P(tpa_dims), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                          ctypes.c_void_p, ctypes.c_void_p]),
     "tpa_get_device_error": (ctypes.c_int, [ctypes.c_void_p, _i32p]),
     "tpa_set_wait_limit": (None, [ctypes.c_uint32]),
 }
@@ -284,6 +287,13 @@ def alloc_step_workspace(dims: Dims, lengths, device="cuda") -> torch.Tensor:
     if n == 0:
         raise ValueError("invalid decode-step arguments")
     return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def tpa_output_project(dims: Dims, attn, w_o, out, stream=None) -> None:
+    """out [T][d_model] = attn [T][h][d_h] (flattened per token) @ w_o[d_model][h*d_h]^T."""
+    T = attn.shape[0]
+    _check("tpa_output_project", _lib.tpa_output_project(ctypes.byref(dims.c()), _ptr(attn), _ptr(w_o),
+                                                         int(T), _ptr(out), _stream(stream)))
 
 
 def tpa_get_device_error(stream=None) -> int:

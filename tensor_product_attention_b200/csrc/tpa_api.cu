@@ -246,6 +246,26 @@ tpa_status tpa_decode(const tpa_dims* d, const void* q_a, const void* q_b,
                       (cudaStream_t)stream);
 }
 
+tpa_status tpa_output_project(const tpa_dims* d, const void* attn, const void* w_o, int32_t T,
+                              void* out, tpa_stream_t stream) {
+    tpa_status st = check_dims(d, false);
+    if (st != TPA_OK) return st;
+    if (d->d_model < 1 || T < 1) return TPA_ERR_INVALID;
+    if (!attn || !w_o || !out) return TPA_ERR_INVALID;
+    if (!aligned16(attn) || !aligned16(w_o) || !aligned16(out)) return TPA_ERR_INVALID;
+    if ((long long)d->n_heads * d->head_dim > (1 << 20) || T > (1 << 30)) return TPA_ERR_UNSUPPORTED;
+    // the projection GEMM with one output segment (no RoPE pair in it): K = h*d_h
+    Shape s = shape_of(*d);
+    s.D = d->n_heads * d->head_dim;
+    ProjLayout L;
+    for (int i = 0; i < 6; ++i) L.off[i] = 0;
+    L.off[6] = d->d_model;
+    for (int i = 0; i < 6; ++i) L.dst[i] = out;
+    SeqParams sp;
+    sp.v[0] = 0;
+    return run_project(s, attn, w_o, 1, T, sp, nullptr, L, (cudaStream_t)stream);
+}
+
 size_t tpa_decode_step_workspace_bytes(const tpa_dims* d, const int32_t* lengths, int32_t batch) {
     if (check_dims(d, false) != TPA_OK || !lengths || batch < 1 || batch > TPA_MAX_BATCH)
         return 0;

@@ -23,7 +23,7 @@ import torch
 
 # stream tags, so that each tensor of a workload has its own random stream
 _TAG = {"x": 1, "w": 2, "len": 3, "a_k": 4, "a_v": 5, "b_k": 6, "b_v": 7,
-        "a_q": 8, "b_q": 9, "q": 10, "misc": 11}
+        "a_q": 8, "b_q": 9, "q": 10, "misc": 11, "wo": 12, "o": 13}
 
 
 @dataclass(frozen=True)
@@ -122,6 +122,19 @@ def prefill_w(wl: Workload, seed: int | None = None) -> torch.Tensor:
     n = sum(factor_widths(wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v))
     g = rng(wl.seed if seed is None else seed, "w")
     return to_storage(normal(g, (n, wl.d_model), 1.0 / np.sqrt(wl.d_model)), wl.dtype)
+
+
+def output_w(wl: Workload, seed: int | None = None) -> torch.Tensor:
+    """The output projection weight: [d_model, n_heads * head_dim] ~ N(0, 1/(h d_h))."""
+    n = wl.n_heads * wl.head_dim
+    g = rng(wl.seed if seed is None else seed, "wo")
+    return to_storage(normal(g, (wl.d_model, n), 1.0 / np.sqrt(n)), wl.dtype)
+
+
+def attn_out(wl: Workload, T: int, seed: int | None = None) -> torch.Tensor:
+    """A stand-in attention output [T, h, d_h] ~ N(0, 1/d_h) (output-projection checks)."""
+    g = rng(wl.seed if seed is None else seed, "o")
+    return to_storage(normal(g, (T, wl.n_heads, wl.head_dim), 1.0 / np.sqrt(wl.head_dim)), wl.dtype)
 
 
 # -------------------------------------------------------------------- decode inputs

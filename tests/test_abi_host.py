@@ -117,6 +117,18 @@ def test_decode_step_host_validation(bnd):
     assert bnd.tpa_decode_step_workspace_bytes(bnd.Dims(64, 4, 16, 2, 1, 1, bnd.F32), [-1]) == 0
 
 
+def test_output_project_host_validation(bnd):
+    d = bnd.Dims(64, 4, 16, 2, 1, 1, bnd.F32).c()
+    by = ctypes.byref
+    fake = 0x10000
+    op = lambda *a: _call(bnd, "tpa_output_project", *a)
+    assert op(by(d), None, fake, 8, fake, None) == 1
+    assert op(by(d), fake, fake, 0, fake, None) == 1
+    assert op(by(d), fake, fake + 4, 8, fake, None) == 1
+    no_model = bnd.Dims(0, 4, 16, 2, 1, 1, bnd.F32).c()
+    assert op(by(no_model), fake, fake, 8, fake, None) == 1
+
+
 def test_workspace_size_formula(bnd):
     dims = bnd.Dims(0, 16, 128, 6, 2, 2)
     lengths = [32768] * 64

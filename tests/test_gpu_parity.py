@@ -365,3 +365,37 @@ def test_decode_step_fused(tpa, case):
     for b, L in enumerate(lengths):
         ref = oracle.tpa_forward_rows(f64(xs[b]), f64(w), od, wl.rope_base, [L])
         assert rel_err(out[b:b + 1], ref) < TOL[wl.dtype], b
+
+
+# ------------------------------------------------------------ output projection
+
+@pytest.mark.parametrize("wl,T", [(TINY, 64), (I.custom("wo_d64", C2, d_model=512), 301),
+                                  (I.custom("wo_d128", C5, d_model=384), 77)],
+                         ids=["f32", "bf16-d64", "bf16-d128"])
+def test_output_project(tpa, wl, T):
+    dims = dims_of(wl, tpa)
+    attn = I.attn_out(wl, T).cuda()
+    w_o = I.output_w(wl).cuda()
+    out = torch.empty((T, wl.d_model), dtype=dims.torch_dtype, device="cuda")
+    tpa.tpa_output_project(dims, attn, w_o, out)
+    torch.cuda.synchronize()
+    assert tpa.tpa_get_device_error() == 0
+    assert rel_err(out, oracle.output_projection(f64(attn), f64(w_o))) < TOL[wl.dtype]
+
+
+def test_full_layer_with_output_projection(tpa):
+    """x -> project -> append -> prefill -> wo, against the pages' forward followed by wo."""
+    wl = I.custom("e_wo", C5, d_model=256)
+    dims = dims_of(wl, tpa)
+    B, S = 2, 90
+    cs = rope_table(tpa, dims, wl.rope_base, S)
+    xs = [I.prefill_x(wl, b, S) for b in range(B)]
+    w, w_o = I.prefill_w(wl), I.output_w(wl)
+    cache = tpa.alloc_cache(dims, B, S)
+    attn = _layer_prefill(tpa, wl, torch.cat(xs).cuda(), w.cuda(), dims, cache, cs, S, [0] * B, S, B)
+    y = torch.empty((B * S, wl.d_model), dtype=torch.bfloat16, device="cuda")
+    tpa.tpa_output_project(dims, attn, w_o.cuda(), y)
+    torch.cuda.synchronize()
+    ref, _ = oracle.tpa_forward(np.stack([f64(xb) for xb in xs]), f64(w), oracle_dims(wl), wl.rope_base)
+    want = oracle.output_projection(ref.reshape(B * S, wl.n_heads, wl.head_dim), f64(w_o))
+    assert rel_err(y, want) < TOL["bf16"]
