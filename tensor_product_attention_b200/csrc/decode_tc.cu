@@ -47,6 +47,7 @@ struct DecodeTcArgs {
     float* ws_ml;                  // [parts][H][2]
     float* ws_o;                   // [parts][H][DH]
     int Rq, cap;
+    int asw;                       // a^K, a^V tiles by TMA with the 128-byte swizzle
     float qscale;
     uint32_t a_bytes, stage_bytes;
     int* err;
@@ -69,6 +70,7 @@ struct TileWalk {
 template <int DH, int HH, int R>
 __global__ void __launch_bounds__(64 + 32 * 4 * (HH / 16), 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                 const __grid_constant__ CUtensorMap tmak, const __grid_constant__ CUtensorMap tmav,
                  const DecodeTcArgs a, const DecodePlan P) {
     constexpr int KT = 128 / R;                 // keys per tile
     constexpr int NB = DH / 64;                 // 64-wide column blocks of d_h (1 or 2)
@@ -124,7 +126,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         *abort = 0;
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) { prefetch_tensormap(&tmk); prefetch_tensormap(&tmv); }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmk); prefetch_tensormap(&tmv);
+        prefetch_tensormap(&tmak); prefetch_tensormap(&tmav);
+    }
     if (warp == 1) { tmem_alloc(tmem_slot, 128); tmem_relinquish(); }
     tc_fence_before();
     __syncthreads();
@@ -146,7 +151,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 if (i >= kStages &&
                     !mbar_wait(&kv_empty[s], (uint32_t)((i / kStages - 1) & 1), lim, a.err, abort))
                     break;
-                const int rows_a = min(KT, a.cap - j0);
+                // a^K, a^V: one TMA box each, 128-byte rows (one key at h 32, two at h 16)
+                // with the 128-byte swizzle; keys past the tensor read as zeros, so the
+                // box lands whole.  Otherwise (odd capacity at h 16) bulk copies.
+                const int rows_a = a.asw ? KT : min(KT, a.cap - j0);
                 const uint32_t abytes = (uint32_t)rows_a * HH * R * 2u;
                 mbar_arrive_expect_tx(&kv_full[s], (NB + 2u) * kBox + 2u * abytes);
                 const int y = (int)(((long long)b * a.cap + j0) * R);
@@ -156,9 +164,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 // loaded twice and output rows 64..127 (a copy of 0..63) are dropped
                 tma_load_2d(st_bv(s), &tmv, &kv_full[s], 0, y);
                 tma_load_2d(st_bv(s) + kBox, &tmv, &kv_full[s], NB == 2 ? 64 : 0, y);
-                const long long ea = ((long long)b * a.cap + j0) * HH * R;
-                bulk_load(st_ak(s), a.ca_k + ea, abytes, &kv_full[s]);
-                bulk_load(st_av(s), a.ca_v + ea, abytes, &kv_full[s]);
+                if (a.asw) {
+                    const int ya = (b * a.cap + j0) / (128 / (HH * R * 2));
+                    tma_load_2d(st_ak(s), &tmak, &kv_full[s], 0, ya);
+                    tma_load_2d(st_av(s), &tmav, &kv_full[s], 0, ya);
+                } else {
+                    const long long ea = ((long long)b * a.cap + j0) * HH * R;
+                    bulk_load(st_ak(s), a.ca_k + ea, abytes, &kv_full[s]);
+                    bulk_load(st_av(s), a.ca_v + ea, abytes, &kv_full[s]);
+                }
             }
             for (int s = 0; s < kStages; ++s) {                 // drain issued copies
                 const int fills = i > s ? (i - s - 1) / kStages + 1 : 0;
@@ -321,12 +335,24 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             // this row's a^K and a^V for the group's 16 heads
             float ak[16], av[16];
             {
-                const __nv_bfloat16* akr = reinterpret_cast<const __nv_bfloat16*>(st_ak(s)) + ((size_t)jl * HH + hbase) * R;
-                const __nv_bfloat16* avr = reinterpret_cast<const __nv_bfloat16*>(st_av(s)) + ((size_t)jl * HH + hbase) * R;
+                static_assert(R == 2, "factor words hold both ranks");
+                // the 32-bit word holds (head, both ranks); this row's rank picks a half.
+                // With the TMA swizzle, 16-byte chunk bits 4..6 are XORed with address bits
+                // 7..9 (the tiles are 1024-aligned), so the 16 keys of a warp spread over
+                // the banks instead of hitting one or two.
+                constexpr uint32_t kRow = HH * R * 2u;
+                const uint32_t kSw = a.asw ? 7u : 0u;
+                const uint32_t akr = smem_u32(st_ak(s)) + (uint32_t)jl * kRow;
+                const uint32_t avr = smem_u32(st_av(s)) + (uint32_t)jl * kRow;
 #pragma unroll
                 for (int h = 0; h < 16; ++h) {
-                    ak[h] = __bfloat162float(akr[h * R + sr]);
-                    av[h] = __bfloat162float(avr[h * R + sr]);
+                    uint32_t ka = akr + (uint32_t)(hbase + h) * 4u, va = avr + (uint32_t)(hbase + h) * 4u;
+                    ka ^= ((ka >> 7) & kSw) << 4;
+                    va ^= ((va >> 7) & kSw) << 4;
+                    const uint32_t kw = lds_u32(ka);
+                    const uint32_t vw = lds_u32(va);
+                    ak[h] = sr ? bf16hi(kw) : bf16lo(kw);
+                    av[h] = sr ? bf16hi(vw) : bf16lo(vw);
                 }
             }
             tmem_ld_wait();
@@ -458,10 +484,28 @@ cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const D
     const uint32_t box[2] = {64, 128};
     if (!make_tmap_bf16(&tmk, c.b_k, 2, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 2, dims, stride, box))
         return cudaErrorInvalidValue;
+    // a^K, a^V as rows of 128 bytes (h R = 64 bf16: one key at h 32, two keys at h 16),
+    // one box of KT keys with the 128-byte swizzle.  Used at h 32, where the per-key
+    // reads of unswizzled rows were 16-way bank conflicts.  At h 16 (8-way) the bulk
+    // copies measured faster (b64 x 32K: 519 against 544 us), so they stay.
+    constexpr int kpr = 128 / (HH * R * 2);      // keys per 128-byte row
+    CUtensorMap tmak, tmav;
+    a.asw = (HH == 32 && c.capacity % kpr == 0) ? 1 : 0;
+    if (a.asw) {
+        const uint64_t adims[2] = {64, (uint64_t)c.batch * c.capacity / kpr};
+        const uint64_t astride[1] = {128};
+        const uint32_t abox[2] = {64, (uint32_t)(KT / kpr)};
+        if (!make_tmap_bf16(&tmak, c.a_k, 2, adims, astride, abox) ||
+            !make_tmap_bf16(&tmav, c.a_v, 2, adims, astride, abox))
+            return cudaErrorInvalidValue;
+    } else {
+        tmak = tmk;     // unused
+        tmav = tmk;
+    }
     constexpr int threads = 64 + 32 * 4 * (HH / 16);
     cudaError_t e = allow_smem(reinterpret_cast<const void*>(decode_tc_kernel<DH, HH, R>), (int)smem);
     if (e != cudaSuccess) return e;
-    decode_tc_kernel<DH, HH, R><<<plan.n_ctas, threads, smem, st>>>(tmk, tmv, a, plan);
+    decode_tc_kernel<DH, HH, R><<<plan.n_ctas, threads, smem, st>>>(tmk, tmv, tmak, tmav, a, plan);
     return cudaGetLastError();
 }
 }  // namespace

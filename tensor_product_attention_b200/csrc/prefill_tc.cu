@@ -106,19 +106,18 @@ __device__ __forceinline__ void softmax_pass(uint32_t u_addr, const __nv_bfloat1
             uint32_t wa[32], wv[32];
             if constexpr (AT) {
                 // ak, av point at this head's transposed rows: 4 keys per 16-byte load
-                const uint4* k4 = reinterpret_cast<const uint4*>(ak);
-                const uint4* v4 = reinterpret_cast<const uint4*>(av);
+                const uint32_t k4 = smem_u32(ak), v4 = smem_u32(av);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const uint4 x = k4[c], y = v4[c];
+                    const uint4 x = lds_v4(k4 + 16u * c), y = lds_v4(v4 + 16u * c);
                     wa[4 * c] = x.x; wa[4 * c + 1] = x.y; wa[4 * c + 2] = x.z; wa[4 * c + 3] = x.w;
                     wv[4 * c] = y.x; wv[4 * c + 1] = y.y; wv[4 * c + 2] = y.z; wv[4 * c + 3] = y.w;
                 }
             } else {
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
-                    wa[q] = akr[q * HS];
-                    wv[q] = avr[q * HS];
+                    wa[q] = lds_u32(smem_u32(akr) + 4u * q * HS);
+                    wv[q] = lds_u32(smem_u32(avr) + 4u * q * HS);
                 }
             }
             tmem_ld_wait();

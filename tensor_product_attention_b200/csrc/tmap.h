@@ -8,10 +8,11 @@
 
 namespace tpa {
 
-// 2-D (or 3-D) bf16 tensor map with 128-byte swizzle; dims/strides innermost first,
+// 2-D (or 3-D) bf16 tensor map, 128-byte swizzle unless swizzle_bytes says 64, 32 or 0;
+// dims/strides innermost first,
 // strides in bytes for dims 1.. .  Returns false if the driver rejects it.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                    const uint64_t* strides_bytes, const uint32_t* box);
+                    const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes = 128);
 
 int sm_count();
 

@@ -181,6 +181,7 @@ DECODE_CASES = [
     (I.custom("d_kvonly", C4), [1, 3001], 8.0),
     # more key tiles than SMs: every CTA walks several tiles, parts cross sequences
     (I.custom("d_multi", C3), [12000, 9001, 1, 14500], 1.0),
+    (I.custom("d_multi", C3), [12000, 9001, 1, 14501], 8.0),
     (I.custom("d_multi", C3), [700] * 29 + [33], 8.0),
     (I.custom("d_kvmulti", C4), [20000, 13001], 8.0),
     # head_dim 64 (the value MMA repeats the 64-wide tile to fill its 128 rows)
