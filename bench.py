@@ -39,6 +39,7 @@ from tensor_product_attention_b200 import inputs as I  # noqa: E402
 METRIC = "TPA decode factor-cache GB/s (% HBM peak); prefill TFLOP/s (% bf16 peak)"
 DEFAULT = "prefill_b8_s2048_d1024"
 DECODE_LEG = "decode_b64_ctx32k"
+KVONLY_DECODE_LEG = "kvonly_decode_b16_ctx64k_128k"
 FLUSH_BYTES = 256 << 20          # > 126 MB L2
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture of
@@ -576,17 +577,20 @@ def main():
     del step
     torch.cuda.empty_cache()
 
-    if wl.kind == "prefill" and not args.no_decode_leg:
-        dl = I.WORKLOADS[DECODE_LEG]
+    # the decode configurations ride along with the prefill step as separate legs
+    legs_to_run = [] if (wl.kind != "prefill" or args.no_decode_leg) else \
+        [("decode_leg", DECODE_LEG), ("kvonly_decode_leg", KVONLY_DECODE_LEG)]
+    for key, name in legs_to_run:
+        dl = I.WORKLOADS[name]
         dstep = DecodeStep(dl, tpa)
         dms = timed(dstep, args.steps, args.warmup, ws, None, graph=not args.no_graph)
         dev = timed_legs(dstep, args.steps, None)
         dval = whole_job_rate(ws, dstep.bytes(), dms) / 1e9
         dach = dstep.factor_bytes() / (dev.mean_ms("decode") * 1e-3) / 1e9
-        line["decode_leg"] = {"workload": dl.name, "value": dval, "unit": "GB/s", "ms_per_step": dms,
-                              "frac_of_hbm": dach / pk["hbm_gbs"], "factor_bytes": dstep.factor_bytes(),
-                              "traffic": PROFILED_TRAFFIC.get((dl.name, "tpa_decode")),
-                              "gpu_launches": dstep.launches_per_step * args.steps}
+        line[key] = {"workload": dl.name, "value": dval, "unit": "GB/s", "ms_per_step": dms,
+                     "frac_of_hbm": dach / pk["hbm_gbs"], "factor_bytes": dstep.factor_bytes(),
+                     "traffic": PROFILED_TRAFFIC.get((dl.name, "tpa_decode")),
+                     "gpu_launches": dstep.launches_per_step * args.steps}
         line["gpu_launches"] += dstep.launches_per_step * args.steps
         del dstep
         torch.cuda.empty_cache()

@@ -341,7 +341,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 // 7..9 (the tiles are 1024-aligned), so the 16 keys of a warp spread over
                 // the banks instead of hitting one or two.
                 constexpr uint32_t kRow = HH * R * 2u;
-                const uint32_t kSw = a.asw ? 7u : 0u;
+                const uint32_t kSw = (HH == 32 && a.asw) ? 7u : 0u;   // folds to 0 at h 16
                 const uint32_t akr = smem_u32(st_ak(s)) + (uint32_t)jl * kRow;
                 const uint32_t avr = smem_u32(st_av(s)) + (uint32_t)jl * kRow;
 #pragma unroll
