@@ -80,6 +80,101 @@ __device__ __forceinline__ void load_r(const __nv_bfloat16* base, int idx, float
     }
 }
 
+// ---- packed path (R = 2, h = 16): the b^K / b^V tiles are loaded rank-major (row
+// s*KT + j), so U and W hold rank 0 of the tile's 32 keys, then rank 1, and two
+// consecutive keys sit in adjacent columns.  The scores of a key pair are then one pair
+// of f32x2 FMAs, p converts to bf16 for both keys at once, and W is two bf16x2 products.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ void lds_v2u64(uint32_t addr, uint64_t& a, uint64_t& b) {
+    asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr));
+}
+
+// Transposed a-factor rows of one head for the packed path: a^K as fp32 [rank][32 keys]
+// (256 B, padded to 272) and a^V as bf16 [rank][32 keys] (128 B, padded to 144).
+constexpr uint32_t kPkPitchK = 272, kPkPitchV = 144;
+
+// One pass over the tile (packed path) for this thread's row (i, h) against m_ref:
+// d_j = a^K_{j,0} U_{0,j} + a^K_{j,1} U_{1,j} - m_ref.  MAXONLY: out = max_j d_j.
+// Otherwise p_j = 2^d_j, out = sum_j p_j, and wp = W in K order (rank, key), packed
+// as bf16 pairs of consecutive keys.  MASKED applies j <= p_i (diagonal tiles).
+template <bool MASKED, bool MAXONLY>
+__device__ __forceinline__ void softmax_pass_pk(const uint32_t (&u)[64], uint32_t akrow, uint32_t avrow,
+                                                int j0, int p_i, float m_ref, float& out,
+                                                uint32_t (&wp)[32]) {
+    const uint64_t mneg = f2pack(-m_ref, -m_ref);
+    uint64_t acc2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
+    float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {                       // 8 keys per chunk
+        uint64_t a0[4], a1[4];
+        lds_v2u64(akrow + 32u * c, a0[0], a0[1]);
+        lds_v2u64(akrow + 32u * c + 16u, a0[2], a0[3]);
+        lds_v2u64(akrow + 128u + 32u * c, a1[0], a1[1]);
+        lds_v2u64(akrow + 128u + 32u * c + 16u, a1[2], a1[3]);
+        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+        if constexpr (!MAXONLY) {
+            v0 = lds_v4(avrow + 16u * c);
+            v1 = lds_v4(avrow + 64u + 16u * c);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int j = 8 * c + 2 * q;
+            const uint64_t u0 = f2pack(__uint_as_float(u[j]), __uint_as_float(u[j + 1]));
+            const uint64_t u1 = f2pack(__uint_as_float(u[32 + j]), __uint_as_float(u[33 + j]));
+            float dl, dh;
+            f2unpack(fma2(a1[q], u1, fma2(a0[q], u0, mneg)), dl, dh);
+            if (MASKED) {
+                dl = (j0 + j <= p_i) ? dl : -INFINITY;
+                dh = (j0 + j + 1 <= p_i) ? dh : -INFINITY;
+            }
+            if constexpr (MAXONLY) {
+                mxa[q] = fmaxf(mxa[q], fmaxf(dl, dh));
+            } else {
+                const float pl = ex2(dl), ph = ex2(dh);
+                acc2[q & 1] = add2(acc2[q & 1], f2pack(pl, ph));
+                const __nv_bfloat162 pb = __floats2bfloat162_rn(pl, ph);
+                const uint32_t av0 = (&v0.x)[q], av1 = (&v1.x)[q];
+                const __nv_bfloat162 w0 = __hmul2(pb, *reinterpret_cast<const __nv_bfloat162*>(&av0));
+                const __nv_bfloat162 w1 = __hmul2(pb, *reinterpret_cast<const __nv_bfloat162*>(&av1));
+                uint32_t x0 = *reinterpret_cast<const uint32_t*>(&w0), x1 = *reinterpret_cast<const uint32_t*>(&w1);
+                if (MASKED) {
+                    // a key past p_i contributes exactly 0 whatever its a^V holds
+                    const uint32_t keep = (pl != 0.f ? 0x0000ffffu : 0u) | (ph != 0.f ? 0xffff0000u : 0u);
+                    x0 &= keep;
+                    x1 &= keep;
+                }
+                wp[4 * c + q] = x0;
+                wp[16 + 4 * c + q] = x1;
+            }
+        }
+    }
+    if constexpr (MAXONLY) {
+        out = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
+    } else {
+        float a0l, a0h, a1l, a1h;
+        f2unpack(acc2[0], a0l, a0h);
+        f2unpack(acc2[1], a1l, a1h);
+        out = (a0l + a0h) + (a1l + a1h);
+    }
+}
+
 // One pass of the softmax over a key tile for this thread's row (i, h), relative to a
 // reference max m_ref: d_j = sum_s a^K_{j,h,s} U_{(j,s)} - m_ref (log2 units), mx =
 // max_j d_j, p_j = 2^d_j, lsum = sum_j p_j, and the W row (p_j a^V_{j,h,s}) in K order
@@ -194,7 +289,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     uint8_t* stg = smem + kQBytes;                        // stages
     // R = 2 at h = 16: warp 3 transposes each tile's a^K, a^V into kATS row-per-head buffers
     constexpr bool AT = R == 2 && HC == 16;
-    constexpr uint32_t kATBytes = AT ? 2u * HC * kATPitch : 0u;       // one transposed tile pair
+    // ... and its softmax runs the packed path on rank-major tiles
+    constexpr bool PK = AT;
+    constexpr uint32_t kATBytes = PK ? HC * (kPkPitchK + kPkPitchV) : AT ? 2u * HC * kATPitch : 0u;
     uint8_t* atr = stg + (size_t)a.stages * a.stage_bytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(atr + kATS * kATBytes);
     uint64_t* kv_full = bars;
@@ -324,8 +421,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 const int y = (int)(((long long)b * a.cap + j0) * R);
 #pragma unroll
                 for (int cb = 0; cb < NB; ++cb) {
-                    tma_load_2d(stage_bk(s) + cb * kBox, &tmk, &kv_full[s], cb * 64, y);
-                    tma_load_2d(stage_bv(s) + cb * kBox, &tmv, &kv_full[s], cb * 64, y);
+                    if constexpr (PK) {
+                        // rank-major box: (column, key, rank) = (cb*64, key of j0, 0)
+                        tma_load_3d(stage_bk(s) + cb * kBox, &tmk, &kv_full[s], cb * 64, b * a.cap + j0, 0);
+                        tma_load_3d(stage_bv(s) + cb * kBox, &tmv, &kv_full[s], cb * 64, b * a.cap + j0, 0);
+                    } else {
+                        tma_load_2d(stage_bk(s) + cb * kBox, &tmk, &kv_full[s], cb * 64, y);
+                        tma_load_2d(stage_bv(s) + cb * kBox, &tmv, &kv_full[s], cb * 64, y);
+                    }
                 }
                 const long long ea = ((long long)b * a.cap + j0) * H * R;
                 bulk_load((void*)stage_ak(s), a.ca_k + ea, abytes, &kv_full[s]);
@@ -421,15 +524,30 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                        mbar_wait(&w_ready[2 + (tp & 1)], (uint32_t)((tp >> 1) & 1), lim, a.err, abort);
             }
             if (__any_sync(0xffffffffu, !good)) break;
-            const uint32_t* sk = reinterpret_cast<const uint32_t*>(stage_ak(s));
-            const uint32_t* sv = reinterpret_cast<const uint32_t*>(stage_av(s));
-            uint32_t* dk = reinterpret_cast<uint32_t*>(atr + (t % kATS) * kATBytes);
-            uint32_t* dv = dk + HC * (kATPitch / 4);
+            const uint32_t sk = smem_u32(stage_ak(s)), sv = smem_u32(stage_av(s));
+            uint8_t* dbase = atr + (t % kATS) * kATBytes;
+            if constexpr (PK) {
+                // a^K as fp32 [head][rank][key], a^V as bf16 [head][rank][key]
+                float* dk = reinterpret_cast<float*>(dbase);
+                uint16_t* dv = reinterpret_cast<uint16_t*>(dbase + HC * kPkPitchK);
 #pragma unroll 4
-            for (int w = lane; w < kWords; w += 32) {
-                const int j = w / HC, hh = w % HC;
-                dk[hh * (kATPitch / 4) + j] = sk[w];
-                dv[hh * (kATPitch / 4) + j] = sv[w];
+                for (int w = lane; w < kWords; w += 32) {
+                    const int j = w / HC, hh = w % HC;
+                    const uint32_t kw = lds_u32(sk + 4u * w), vw = lds_u32(sv + 4u * w);
+                    dk[hh * (kPkPitchK / 4) + j] = bf16lo(kw);
+                    dk[hh * (kPkPitchK / 4) + 32 + j] = bf16hi(kw);
+                    dv[hh * (kPkPitchV / 2) + j] = (uint16_t)(vw & 0xffffu);
+                    dv[hh * (kPkPitchV / 2) + 32 + j] = (uint16_t)(vw >> 16);
+                }
+            } else {
+                uint32_t* dk = reinterpret_cast<uint32_t*>(dbase);
+                uint32_t* dv = dk + HC * (kATPitch / 4);
+#pragma unroll 4
+                for (int w = lane; w < kWords; w += 32) {
+                    const int j = w / HC, hh = w % HC;
+                    dk[hh * (kATPitch / 4) + j] = lds_u32(sk + 4u * w);
+                    dv[hh * (kATPitch / 4) + j] = lds_u32(sv + 4u * w);
+                }
             }
             mbar_arrive(&at_ready[t % kATS]);
             if (++s == a.stages) { s = 0; ph ^= 1u; }
@@ -472,6 +590,52 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             uint32_t wp[32];
             float mx = -INFINITY, lsum = 0.f;
             bool ok = false;
+            if constexpr (PK) {
+                uint32_t u[64];
+                tmem_ld32(u_addr, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+                tmem_ld32(u_addr + 32u, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+                const uint32_t akrow = smem_u32(atr + (t % kATS) * kATBytes) + (uint32_t)h * kPkPitchK;
+                const uint32_t avrow = smem_u32(atr + (t % kATS) * kATBytes + HC * kPkPitchK) + (uint32_t)h * kPkPitchV;
+                tmem_ld_wait();
+                if (t > 0) {
+                    // one pass against the running max; if the tile's sum stays within
+                    // 2^8, so does every term, and no rescale is needed
+                    if (masked) softmax_pass_pk<true, false>(u, akrow, avrow, j0, p_i, m_use, lsum, wp);
+                    else softmax_pass_pk<false, false>(u, akrow, avrow, j0, p_i, m_use, lsum, wp);
+                    ok = lsum <= 256.f;
+                }
+                if (__all_sync(0xffffffffu, ok)) {
+                    l += lsum;
+                } else {
+                    // first tile, or a score well above the running max: exact max, rescale O
+                    const float m_ref = t == 0 ? 0.f : m_use;
+                    if (masked) softmax_pass_pk<true, true>(u, akrow, avrow, j0, p_i, m_ref, mx, wp);
+                    else softmax_pass_pk<false, true>(u, akrow, avrow, j0, p_i, m_ref, mx, wp);
+                    const float m_new = t == 0 ? mx : m_use + fmaxf(mx, 0.f);
+                    const float alpha = t == 0 ? 1.f : ex2(m_use - m_new);
+                    if (t > 0) l *= alpha;
+                    if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                        // O row *= alpha, once PV(t-1) into O has completed
+                        const bool pv_done = mbar_wait(&o_ready[bl], (uint32_t)((t - 1) & 1), lim, a.err, abort);
+                        if (__any_sync(0xffffffffu, !pv_done)) { alive = false; break; }
+                        tc_fence_after();
+#pragma unroll
+                        for (int c = 0; c < DH / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(lane_addr + o_col + (uint32_t)c * 32u, o);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                            tmem_st32(lane_addr + o_col + (uint32_t)c * 32u, o);
+                        }
+                        tmem_st_wait();
+                    }
+                    m_use = m_new;
+                    if (masked) softmax_pass_pk<true, false>(u, akrow, avrow, j0, p_i, m_use, lsum, wp);
+                    else softmax_pass_pk<false, false>(u, akrow, avrow, j0, p_i, m_use, lsum, wp);
+                    l += lsum;
+                }
+            } else {
             if (t > 0) {
                 // common case: one pass against the running max
                 if (masked) softmax_pass<R, true, HC, AT>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
@@ -510,20 +674,25 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 else softmax_pass<R, false, HC, AT>(u_addr, ak, av, H, h, j0, p_i, m_use, mx, lsum, wp);
                 l += lsum;
             }
+            }
             // W over the first half of U (the scores have all been read)
             tmem_st32(u_addr, wp);
             tmem_st_wait();
             if (bl == 0 && t == n_tiles - 1 && j0 + KT > kv_len) {
                 // keys at or past the valid length: clear their b^V rows so that
                 // 0 * (whatever the cache holds there) stays 0 in the PV product
+                // (tile rows are (key, rank), or rank-major s*KT + key on the packed path)
                 uint8_t* bv = stage_bv(s);
-                const int first = (kv_len - j0) * R;
-                for (int rr = first + (threadIdx.x - 128); rr < UW; rr += 128)
+                const int nv = kv_len - j0;                 // valid keys in the tile
+                for (int idx = threadIdx.x - 128; idx < UW; idx += 128) {
+                    const int key = PK ? idx % KT : idx / R;
+                    if (key < nv) continue;
                     for (int cb = 0; cb < NB; ++cb) {
-                        uint4* pz = reinterpret_cast<uint4*>(bv + cb * kBox + rr * 128);
+                        uint4* pz = reinterpret_cast<uint4*>(bv + cb * kBox + idx * 128);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) pz[e] = make_uint4(0, 0, 0, 0);
                     }
+                }
                 fence_proxy_async_smem();
             }
             tc_fence_before();
@@ -572,16 +741,26 @@ cudaError_t launch_t(const PrefillTcArgs& a0, const tpa_cache& c, int batch, con
     const uint32_t a_pad = (a.a_bytes + 127u) & ~127u;
     a.stage_bytes = ((2u * NB * kBox + 2u * a_pad) + 1023u) & ~1023u;
     const uint32_t q_bytes = DH == 64 ? 0u : NB * 256u * 128u;   // q~ in TMEM at d_h 64
-    const uint32_t at_bytes = (R == 2 && HC == 16) ? kATS * 2u * HC * kATPitch : 0u;
+    const uint32_t at_bytes = (R == 2 && HC == 16) ? kATS * HC * (kPkPitchK + kPkPitchV) : 0u;
     const uint32_t budget = 227u * 1024u - 1024u - 512u - q_bytes - at_bytes;
     a.stages = std::min(8, (int)(budget / a.stage_bytes));
     if (a.stages < 3) return cudaErrorInvalidValue;   // QK(t+2) and PV(t) use different stages
     CUtensorMap tmk, tmv;
-    const uint64_t dims[2] = {(uint64_t)DH, (uint64_t)c.batch * c.capacity * R};
-    const uint64_t stride[1] = {(uint64_t)DH * 2};
-    const uint32_t box[2] = {64, (uint32_t)kUW};
-    if (!make_tmap_bf16(&tmk, c.b_k, 2, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 2, dims, stride, box))
-        return cudaErrorInvalidValue;
+    if constexpr (R == 2 && HC == 16) {
+        // packed path: [d_h][key][rank] with rank outermost, so a box of KT keys x 2
+        // ranks lands rank-major (row s*KT + key)
+        const uint64_t dims[3] = {(uint64_t)DH, (uint64_t)c.batch * c.capacity, (uint64_t)R};
+        const uint64_t stride[2] = {(uint64_t)R * DH * 2, (uint64_t)DH * 2};
+        const uint32_t box[3] = {64, (uint32_t)KT, (uint32_t)R};
+        if (!make_tmap_bf16(&tmk, c.b_k, 3, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 3, dims, stride, box))
+            return cudaErrorInvalidValue;
+    } else {
+        const uint64_t dims[2] = {(uint64_t)DH, (uint64_t)c.batch * c.capacity * R};
+        const uint64_t stride[1] = {(uint64_t)DH * 2};
+        const uint32_t box[2] = {64, (uint32_t)kUW};
+        if (!make_tmap_bf16(&tmk, c.b_k, 2, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 2, dims, stride, box))
+            return cudaErrorInvalidValue;
+    }
     const size_t smem = 1024 + q_bytes + (size_t)a.stages * a.stage_bytes + at_bytes + (2 * a.stages + 14 + kATS) * 8 + 16;
     cudaError_t e = allow_smem(reinterpret_cast<const void*>(prefill_tc_kernel<DH, R, HC>), (int)smem);
     if (e != cudaSuccess) return e;
@@ -602,7 +781,7 @@ bool prefill_tc_supported(const Shape& s) {
     const uint32_t nb = (uint32_t)s.Dh / 64u;
     const uint32_t a_pad = (128u * (uint32_t)s.H + 127u) & ~127u;
     const uint32_t stage = ((2u * nb * kBox + 2u * a_pad) + 1023u) & ~1023u;
-    const uint32_t at_bytes = (s.Rk == 2 && s.H == 16) ? kATS * 2u * 16u * kATPitch : 0u;
+    const uint32_t at_bytes = (s.Rk == 2 && s.H == 16) ? kATS * 16u * (kPkPitchK + kPkPitchV) : 0u;
     return 227u * 1024u - 1024u - 512u - nb * 256u * 128u - at_bytes >= 3u * stage;
 }
 
