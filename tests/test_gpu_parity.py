@@ -133,6 +133,11 @@ PREFILL_CASES = [
     (I.custom("p_d128", C5), 2, 150, [0, 90], 1.0),
     (I.custom("p_d128", C5), 1, 1, [300], 8.0),
     (I.custom("p_d128", C5), 1, 256, [0], 8.0),
+    # the tensor-core kernel's generic paths: ranks 1 and 4, head counts other than 16
+    (I.custom("p_r1", C2, n_heads=8, rank_k=1, rank_v=1, rank_q=3), 2, 150, [0, 40], 8.0),
+    (I.custom("p_r4", C2, rank_k=4, rank_v=4), 2, 97, [5, 0], 8.0),
+    (I.custom("p_h32", C5, n_heads=32), 1, 160, [30], 8.0),
+    (I.custom("p_h4", C2, n_heads=4, rank_k=2, rank_v=2), 1, 300, [0], 1.0),
     # TPA-KVonly: plain per-head query (rank_q = 0)
     (I.custom("p_kv_f32", C4, dtype="f32", n_heads=4, head_dim=32), 2, 45, [0, 20], 8.0),
     (I.custom("p_kv_d128", C4, n_heads=16), 2, 170, [0, 33], 1.0),
