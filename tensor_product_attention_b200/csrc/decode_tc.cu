@@ -37,7 +37,7 @@ using namespace sm100;
 
 constexpr uint32_t kBox = 128 * 128;     // one TMA box: 128 rows x 128 bytes
 constexpr float kTau = 8.f;              // lazy rescale threshold (log2 units)
-constexpr int kStages = 2;
+constexpr int kVS = 2;                   // V ring depth (b^V tiles, read by PV)
 
 struct DecodeTcArgs {
     const __nv_bfloat16* q_a;      // [B][H][Rq] or null
@@ -49,7 +49,8 @@ struct DecodeTcArgs {
     int Rq, cap;
     int asw;                       // a^K, a^V tiles by TMA with the 128-byte swizzle
     float qscale;
-    uint32_t a_bytes, stage_bytes;
+    uint32_t a_bytes, kstage_bytes;  // a^K (or a^V) tile; one K-ring stage (b^K, a^K, a^V)
+    int ks;                          // K ring depth (2..4, as shared memory allows)
     int* err;
     uint32_t wait_limit;
 };
@@ -68,7 +69,7 @@ struct TileWalk {
 };
 
 template <int DH, int HH, int R>
-__global__ void __launch_bounds__(64 + 32 * 4 * (HH / 16), 1)
+__global__ void __launch_bounds__(96 + 32 * 4 * (HH / 16), 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                  const __grid_constant__ CUtensorMap tmak, const __grid_constant__ CUtensorMap tmav,
                  const DecodeTcArgs a, const DecodePlan P) {
@@ -81,14 +82,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint8_t* stg = smem;                                            // kStages stages
-    uint8_t* qbuf = stg + (size_t)kStages * a.stage_bytes;          // 2 x q~
+    // Two rings: K (b^K, a^K, a^V: read by QK and the softmax) a.ks deep, and V (b^V:
+    // read by PV) kVS deep, so the key side prefetches further than the value side.
+    uint8_t* kring = smem;
+    uint8_t* vring = kring + (size_t)a.ks * a.kstage_bytes;
+    uint8_t* qbuf = vring + (size_t)kVS * 2 * kBox;                 // 2 x q~
     uint8_t* wbuf = qbuf + 2 * kQW;                                 // 2 x W^T
     float* red = reinterpret_cast<float*>(wbuf + 2 * kQW);          // [NG][4][16] scratch
     uint64_t* bars = reinterpret_cast<uint64_t*>(red + NG * 64);
-    uint64_t* kv_full = bars;                    // [kStages]
-    uint64_t* kv_empty = kv_full + kStages;      // [kStages]
-    uint64_t* u_full = kv_empty + kStages;       // [2]
+    uint64_t* k_full = bars;                     // [ks]
+    uint64_t* k_empty = k_full + a.ks;           // [ks] every softmax thread is done with it
+    uint64_t* v_full = k_empty + a.ks;           // [kVS]
+    uint64_t* v_empty = v_full + kVS;            // [kVS] its PV has completed
+    uint64_t* u_full = v_empty + kVS;            // [2]
     uint64_t* w_full = u_full + 2;               // [2]
     uint64_t* w_empty = w_full + 2;              // [2]
     uint64_t* q_ready = w_empty + 2;             // [2]
@@ -98,12 +104,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-    auto st_bk = [&](int s) { return stg + (size_t)s * a.stage_bytes; };
-    auto st_bv = [&](int s) { return stg + (size_t)s * a.stage_bytes + 2 * kBox; };
-    auto st_ak = [&](int s) { return stg + (size_t)s * a.stage_bytes + 4 * kBox; };
+    auto st_bk = [&](int s) { return kring + (size_t)s * a.kstage_bytes; };
+    auto st_ak = [&](int s) { return kring + (size_t)s * a.kstage_bytes + NB * kBox; };
     auto st_av = [&](int s) {
-        return stg + (size_t)s * a.stage_bytes + 4 * kBox + ((a.a_bytes + 127u) & ~127u);
+        return kring + (size_t)s * a.kstage_bytes + NB * kBox + ((a.a_bytes + 127u) & ~127u);
     };
+    auto st_bv = [&](int s) { return vring + (size_t)s * 2 * kBox; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x;
@@ -113,7 +119,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     const uint32_t lim = a.wait_limit;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+        for (int s = 0; s < a.ks; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], NSM); }
+        for (int s = 0; s < kVS; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&u_full[i], 1);
             mbar_init(&w_full[i], NSM);
@@ -136,8 +143,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ---------------------------------------------------------------- producer
+    if (warp == 0 || warp == 2) {
+        // ---------------------------------------------------------------- producers
+        // warp 0: the K ring (b^K, a^K, a^V); warp 2: the V ring (b^V)
+        const bool kside = warp == 0;
+        const int depth = kside ? a.ks : kVS;
+        uint64_t* full = kside ? k_full : v_full;
+        uint64_t* empty = kside ? k_empty : v_empty;
         if (lane == 0 && n > 0) {
             TileWalk<KT> tw;
             tw.init(P, g0);
@@ -147,37 +159,41 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 tw.advance(P, g);
                 const int b = tw.b;
                 const int j0 = (g - P.tile_prefix[b]) * KT;
-                const int s = i % kStages;
-                if (i >= kStages &&
-                    !mbar_wait(&kv_empty[s], (uint32_t)((i / kStages - 1) & 1), lim, a.err, abort))
+                const int s = i % depth;
+                if (i >= depth &&
+                    !mbar_wait(&empty[s], (uint32_t)((i / depth - 1) & 1), lim, a.err, abort))
                     break;
-                // a^K, a^V: one TMA box each, 128-byte rows (one key at h 32, two at h 16)
-                // with the 128-byte swizzle; keys past the tensor read as zeros, so the
-                // box lands whole.  Otherwise (odd capacity at h 16) bulk copies.
-                const int rows_a = a.asw ? KT : min(KT, a.cap - j0);
-                const uint32_t abytes = (uint32_t)rows_a * HH * R * 2u;
-                mbar_arrive_expect_tx(&kv_full[s], (NB + 2u) * kBox + 2u * abytes);
                 const int y = (int)(((long long)b * a.cap + j0) * R);
-                tma_load_2d(st_bk(s), &tmk, &kv_full[s], 0, y);
-                if (NB == 2) tma_load_2d(st_bk(s) + kBox, &tmk, &kv_full[s], 64, y);
-                // the value MMA has M = 128 rows of d_h: for d_h = 64 the one box is
-                // loaded twice and output rows 64..127 (a copy of 0..63) are dropped
-                tma_load_2d(st_bv(s), &tmv, &kv_full[s], 0, y);
-                tma_load_2d(st_bv(s) + kBox, &tmv, &kv_full[s], NB == 2 ? 64 : 0, y);
-                if (a.asw) {
-                    const int ya = (b * a.cap + j0) / (128 / (HH * R * 2));
-                    tma_load_2d(st_ak(s), &tmak, &kv_full[s], 0, ya);
-                    tma_load_2d(st_av(s), &tmav, &kv_full[s], 0, ya);
+                if (kside) {
+                    // a^K, a^V: one TMA box each, 128-byte rows (one key at h 32, two at
+                    // h 16) with the 128-byte swizzle; keys past the tensor read as zeros,
+                    // so the box lands whole.  Otherwise (h 16) bulk copies of the valid rows.
+                    const int rows_a = a.asw ? KT : min(KT, a.cap - j0);
+                    const uint32_t abytes = (uint32_t)rows_a * HH * R * 2u;
+                    mbar_arrive_expect_tx(&full[s], NB * kBox + 2u * abytes);
+                    tma_load_2d(st_bk(s), &tmk, &full[s], 0, y);
+                    if (NB == 2) tma_load_2d(st_bk(s) + kBox, &tmk, &full[s], 64, y);
+                    if (a.asw) {
+                        const int ya = (b * a.cap + j0) / (128 / (HH * R * 2));
+                        tma_load_2d(st_ak(s), &tmak, &full[s], 0, ya);
+                        tma_load_2d(st_av(s), &tmav, &full[s], 0, ya);
+                    } else {
+                        const long long ea = ((long long)b * a.cap + j0) * HH * R;
+                        bulk_load(st_ak(s), a.ca_k + ea, abytes, &full[s]);
+                        bulk_load(st_av(s), a.ca_v + ea, abytes, &full[s]);
+                    }
                 } else {
-                    const long long ea = ((long long)b * a.cap + j0) * HH * R;
-                    bulk_load(st_ak(s), a.ca_k + ea, abytes, &kv_full[s]);
-                    bulk_load(st_av(s), a.ca_v + ea, abytes, &kv_full[s]);
+                    // the value MMA has M = 128 rows of d_h: for d_h = 64 the one box is
+                    // loaded twice and output rows 64..127 (a copy of 0..63) are dropped
+                    mbar_arrive_expect_tx(&full[s], 2u * kBox);
+                    tma_load_2d(st_bv(s), &tmv, &full[s], 0, y);
+                    tma_load_2d(st_bv(s) + kBox, &tmv, &full[s], NB == 2 ? 64 : 0, y);
                 }
             }
-            for (int s = 0; s < kStages; ++s) {                 // drain issued copies
-                const int fills = i > s ? (i - s - 1) / kStages + 1 : 0;
+            for (int s = 0; s < depth; ++s) {                   // drain issued copies
+                const int fills = i > s ? (i - s - 1) / depth + 1 : 0;
                 if (fills > 0)
-                    drain_wait(&kv_full[s], (uint32_t)((fills - 1) & 1));
+                    drain_wait(&full[s], (uint32_t)((fills - 1) & 1));
             }
         }
     } else if (warp == 1) {
@@ -202,8 +218,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 if (first && segp > 0 &&
                     !mbar_wait(o_free, (uint32_t)((segp - 1) & 1), lim, a.err, abort))
                     return false;
+                const int s = j % kVS;
+                if (!mbar_wait(&v_full[s], (uint32_t)((j / kVS) & 1), lim, a.err, abort)) return false;
                 tc_fence_after();
-                const int s = j % kStages;
                 const uint32_t bv = smem_u32(st_bv(s));
                 const uint32_t wb = w0 + (uint32_t)(j & 1) * kQW;
 #pragma unroll
@@ -214,7 +231,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                            idesc_pv, (first && k == 0) ? 0u : 1u);
                 }
                 mma_commit(&w_empty[j & 1]);
-                mma_commit(&kv_empty[s]);
+                mma_commit(&v_empty[s]);
                 if (last) mma_commit(o_done);
                 return true;
             };
@@ -234,8 +251,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                         prev_bq = twq.b;
                         if (!mbar_wait(&q_ready[segq & 1], (uint32_t)((segq >> 1) & 1), lim, a.err, abort)) break;
                     }
-                    const int s = i % kStages;
-                    if (!mbar_wait(&kv_full[s], (uint32_t)((i / kStages) & 1), lim, a.err, abort)) break;
+                    const int s = i % a.ks;
+                    if (!mbar_wait(&k_full[s], (uint32_t)((i / a.ks) & 1), lim, a.err, abort)) break;
                     tc_fence_after();
                     const uint32_t bk = smem_u32(st_bk(s));
                     const uint32_t qb = q0 + (uint32_t)(segq & 1) * kQW;
@@ -257,12 +274,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         }
     } else {
         // ---------------------------------------------------------------- softmax
-        const int sw = warp - 2;                 // 0 .. 4*NG-1
+        const int sw = warp - 3;                 // 0 .. 4*NG-1
         const int hg = sw >> 2;                  // head group (16 heads)
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;       // TMEM lane = tile row (key j, rank s)
         const int jl = r / R, sr = r % R;
-        const int stid = threadIdx.x - 64;       // 0 .. NSM-1
+        const int stid = threadIdx.x - 96;       // 0 .. NSM-1
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
         const int hbase = hg * 16;
         float m[16], lp[16];
@@ -326,9 +343,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             const int j0 = (g - P.tile_prefix[b]) * KT;
             const int len = P.len[b];
             const bool valid = j0 + jl < len;
-            const int s = i % kStages;
+            const int s = i % a.ks;
             if (!bad) bad = !mbar_wait(&u_full[i & 1], (uint32_t)((i >> 1) & 1), lim, a.err, abort);
-            if (!bad) bad = !mbar_wait(&kv_full[s], (uint32_t)((i / kStages) & 1), lim, a.err, abort);
+            if (!bad) bad = !mbar_wait(&k_full[s], (uint32_t)((i / a.ks) & 1), lim, a.err, abort);
             tc_fence_after();
             uint32_t u[16];
             tmem_ld16(lane_addr + (uint32_t)(i & 1) * HH + hbase, u);
@@ -418,15 +435,21 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 }
             }
             if (hg == 0 && !valid && j0 + jl >= len) {
-                // keys past the sequence: clear their b^V row so 0 * (cache contents) = 0
-                uint4* z0 = reinterpret_cast<uint4*>(st_bv(s) + r * 128);
-                uint4* z1 = reinterpret_cast<uint4*>(st_bv(s) + kBox + r * 128);
+                // keys past the sequence: clear their b^V row (once the tile has landed)
+                // so 0 * (cache contents) = 0
+                const int sv = i % kVS;
+                if (!bad) bad = !mbar_wait(&v_full[sv], (uint32_t)((i / kVS) & 1), lim, a.err, abort);
+                if (!bad) {
+                    uint4* z0 = reinterpret_cast<uint4*>(st_bv(sv) + r * 128);
+                    uint4* z1 = reinterpret_cast<uint4*>(st_bv(sv) + kBox + r * 128);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) { z0[e] = make_uint4(0, 0, 0, 0); z1[e] = make_uint4(0, 0, 0, 0); }
+                    for (int e = 0; e < 8; ++e) { z0[e] = make_uint4(0, 0, 0, 0); z1[e] = make_uint4(0, 0, 0, 0); }
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&w_full[i & 1]);
+            mbar_arrive(&k_empty[s]);                // this thread is done with the K stage
             const bool last = (i == n - 1) || (P.tile_prefix[b + 1] <= g + 1);
             if (last) {
                 // part done: O^T (lane = d row), l per head, written to the workspace
@@ -474,9 +497,12 @@ cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const D
     constexpr int KT = 128 / R;
     a.a_bytes = (uint32_t)(KT * HH * R * 2);
     const uint32_t a_pad = (a.a_bytes + 127u) & ~127u;
-    a.stage_bytes = ((4u * kBox + 2u * a_pad) + 1023u) & ~1023u;
-    const size_t smem = 1024 + (size_t)kStages * a.stage_bytes + 4u * HH * 256u +
-                        (HH / 16) * 64 * sizeof(float) + 32 * 8 + 16;
+    constexpr int NB = DH / 64;
+    a.kstage_bytes = ((NB * kBox + 2u * a_pad) + 1023u) & ~1023u;
+    const size_t fixed = 1024 + (size_t)kVS * 2 * kBox + 4u * HH * 256u + (HH / 16) * 64 * sizeof(float) + 32 * 8 + 16;
+    a.ks = 4;
+    while (a.ks > 2 && fixed + (size_t)a.ks * a.kstage_bytes > 227 * 1024) --a.ks;
+    const size_t smem = fixed + (size_t)a.ks * a.kstage_bytes;
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
     CUtensorMap tmk, tmv;
     const uint64_t dims[2] = {(uint64_t)DH, (uint64_t)c.batch * c.capacity * R};
@@ -502,7 +528,7 @@ cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const D
         tmak = tmk;     // unused
         tmav = tmk;
     }
-    constexpr int threads = 64 + 32 * 4 * (HH / 16);
+    constexpr int threads = 96 + 32 * 4 * (HH / 16);
     cudaError_t e = allow_smem(reinterpret_cast<const void*>(decode_tc_kernel<DH, HH, R>), (int)smem);
     if (e != cudaSuccess) return e;
     decode_tc_kernel<DH, HH, R><<<plan.n_ctas, threads, smem, st>>>(tmk, tmv, tmak, tmav, a, plan);
