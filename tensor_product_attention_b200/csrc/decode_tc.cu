@@ -358,7 +358,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 // 7..9 (the tiles are 1024-aligned), so the 16 keys of a warp spread over
                 // the banks instead of hitting one or two.
                 constexpr uint32_t kRow = HH * R * 2u;
-                const uint32_t kSw = (HH == 32 && a.asw) ? 7u : 0u;   // folds to 0 at h 16
+                const uint32_t kSw = a.asw ? 7u : 0u;
                 const uint32_t akr = smem_u32(st_ak(s)) + (uint32_t)jl * kRow;
                 const uint32_t avr = smem_u32(st_av(s)) + (uint32_t)jl * kRow;
 #pragma unroll
@@ -511,12 +511,12 @@ cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const D
     if (!make_tmap_bf16(&tmk, c.b_k, 2, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 2, dims, stride, box))
         return cudaErrorInvalidValue;
     // a^K, a^V as rows of 128 bytes (h R = 64 bf16: one key at h 32, two keys at h 16),
-    // one box of KT keys with the 128-byte swizzle.  Used at h 32, where the per-key
-    // reads of unswizzled rows were 16-way bank conflicts.  At h 16 (8-way) the bulk
-    // copies measured faster (b64 x 32K: 519 against 544 us), so they stay.
+    // one box of KT keys with the 128-byte swizzle: the per-key reads of unswizzled rows
+    // were 16-way (h 32) and 8-way (h 16) bank conflicts.  At h 16 a row holds two keys,
+    // so the capacity must be even (else bulk copies).
     constexpr int kpr = 128 / (HH * R * 2);      // keys per 128-byte row
     CUtensorMap tmak, tmav;
-    a.asw = (HH == 32 && c.capacity % kpr == 0) ? 1 : 0;
+    a.asw = (c.capacity % kpr == 0) ? 1 : 0;
     if (a.asw) {
         const uint64_t adims[2] = {64, (uint64_t)c.batch * c.capacity / kpr};
         const uint64_t astride[1] = {128};
