@@ -48,7 +48,7 @@ FLUSH_BYTES = 256 << 20          # > 126 MB L2
 # sequences and scaled by the keys processed (traffic grows in proportion).
 PROFILED_TRAFFIC = {
     ("prefill_b8_s2048_d1024", "tpa_prefill"): 26.45e6 + 0.084e6,
-    ("decode_b64_ctx32k", "tpa_decode"): 4 * (604.10e6 + 5.49e6),
+    ("decode_b64_ctx32k", "tpa_decode"): 4 * (604.10e6 + 5.88e6),
 }
 
 
