@@ -43,6 +43,12 @@ class Dims:
     d_model = ``dim``, n_heads = ``n_heads``, head_dim = ``head_dim``, rank_q =
     ``q_rank``; the page uses one ``rank`` for K and V, kept here as rank_k = rank_v.
     rank_q = 0 marks the TPA-KVonly variant, whose query is a plain per-head vector.
+    shared_basis marks the variant whose key and value B factors are shared across
+    tokens ([review] 优点与创新 5, "跨标记共享基向量"): the pages name it in one clause.
+    Reading taken: B_K and B_V are layer parameters, b_r^K(x_t) = b_r^K for every token
+    (the non-contextual B of 优点与创新 4 applied to B), A_K and A_V stay contextual, the
+    query keeps its own factors, and RoPE acts on the key at its position as in
+    contextual TPA.  The per-token projections W_B_k, W_B_v then do not exist.
     """
 
     d_model: int
@@ -51,6 +57,7 @@ class Dims:
     rank_q: int
     rank_k: int
     rank_v: int
+    shared_basis: bool = False
 
 
 def factor_widths(dims: Dims) -> dict:
@@ -60,23 +67,27 @@ def factor_widths(dims: Dims) -> dict:
     TPA-KVonly (rank_q = 0) keeps the standard query projection ([review] 实验/结果
     names the variant; its projection is not printed).  Reading taken: it takes the
     b_q slot as W_Q with n_heads*head_dim outputs, viewed (n_heads, head_dim), and the
-    a_q slot is empty."""
+    a_q slot is empty.  With a shared basis the b_k and b_v slots are empty (their
+    factors are parameters, not projections of x_t)."""
     h, d = dims.n_heads, dims.head_dim
     return {
         "a_q": h * dims.rank_q,
         "a_k": h * dims.rank_k,
         "a_v": h * dims.rank_v,
         "b_q": (dims.rank_q if dims.rank_q > 0 else h) * d,
-        "b_k": dims.rank_k * d,
-        "b_v": dims.rank_v * d,
+        "b_k": 0 if dims.shared_basis else dims.rank_k * d,
+        "b_v": 0 if dims.shared_basis else dims.rank_v * d,
     }
 
 
 def cache_elements_per_token(dims: Dims) -> int:
     """Factor-cache elements stored per token: cache_kA/cache_vA are [.., n_heads, rank]
     and cache_kB/cache_vB are [.., rank, head_dim] ([review] 类定义与初始化), i.e.
-    (R_K + R_V) * (h + d_h)."""
+    (R_K + R_V) * (h + d_h).  With a shared basis only the A factors are per token:
+    (R_K + R_V) * h."""
     h, d = dims.n_heads, dims.head_dim
+    if dims.shared_basis:
+        return dims.rank_k * h + dims.rank_v * h
     return dims.rank_k * h + dims.rank_v * h + dims.rank_k * d + dims.rank_v * d
 
 
@@ -142,6 +153,8 @@ def split_factors(y: np.ndarray, dims: Dims) -> dict:
         if dims.rank_q == 0 and name in ("a_q", "b_q"):
             if name == "b_q":
                 out["q"] = part.reshape(lead + (h, d))     # TPA-KVonly: the plain query
+        elif w == 0 and name in ("b_k", "b_v"):
+            pass                                           # shared basis: not projected
         elif name.startswith("a_"):
             out[name] = part.reshape(lead + (h, r))
         else:
@@ -205,8 +218,30 @@ def causal_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
     return out
 
 
+def broadcast_basis(basis: dict, n_tokens: int, dims: Dims) -> dict:
+    """The shared-basis variant's B_K and B_V for ``n_tokens`` tokens: every token's
+    factor is the layer's basis, b_r(x_t) = b_r ([review] 优点与创新 5, reading in
+    ``Dims``).  basis["b_k"]: [R_K, d], basis["b_v"]: [R_V, d] -> [n_tokens, R, d]."""
+    out = {}
+    for n, r in (("b_k", dims.rank_k), ("b_v", dims.rank_v)):
+        b = np.asarray(basis[n], dtype=np.float64).reshape(r, dims.head_dim)
+        out[n] = np.broadcast_to(b, (n_tokens, r, dims.head_dim))
+    return out
+
+
+def shared_basis_tables(basis: dict, dims: Dims, capacity: int, rope_base: float) -> dict:
+    """The shared-basis cache's B side for positions 0..capacity-1, pre-rotated as
+    contextual TPA caches B_K ([review] 关键问题及回答 问题2): row p of b_k is the key
+    basis rotated at position p, row p of b_v is the value basis (no rotation).  Every
+    sequence's key at position p uses row p, so these are per layer, not per sequence.
+    Returns {"b_k": [capacity, R_K, d], "b_v": [capacity, R_V, d]}."""
+    b = broadcast_basis(basis, capacity, dims)
+    return {"b_k": rope_rotate(b["b_k"], np.arange(capacity), rope_base),
+            "b_v": np.array(b["b_v"])}
+
+
 def tpa_forward(x: np.ndarray, w_cat: np.ndarray, dims: Dims, rope_base: float,
-                start_pos: int = 0, prior: dict | None = None):
+                start_pos: int = 0, prior: dict | None = None, basis: dict | None = None):
     """The pages' TPA forward for one batch, without the output projection.
 
     Follows [review] 前向传播 in the page's own order: project x into the six
@@ -215,7 +250,8 @@ def tpa_forward(x: np.ndarray, w_cat: np.ndarray, dims: Dims, rope_base: float,
     cache back over [0, start_pos+S); materialise q, k, v with bmm and 1/R; apply
     RoPE to the materialised q (positions start_pos+i) and k (positions j); causal
     softmax attention.  ``self.wo`` is not applied: the page uses it without defining
-    it in __init__.
+    it in __init__.  With a shared basis (``dims.shared_basis``) ``basis`` holds the
+    layer's b_k [R_K, d] and b_v [R_V, d], used as every token's B_K and B_V.
 
     x: [B, S, d_model].  Returns (out [B, S, h, d], new) where ``new`` holds the
     un-rotated factors of the S new tokens ([B, S, ...] each).
@@ -224,13 +260,16 @@ def tpa_forward(x: np.ndarray, w_cat: np.ndarray, dims: Dims, rope_base: float,
     B, S, _ = x.shape
     new = project(x.reshape(B * S, -1), w_cat, dims)
     new = {n: t.reshape((B, S) + t.shape[1:]) for n, t in new.items()}
+    cached = ("a_k", "a_v") if dims.shared_basis else ("a_k", "a_v", "b_k", "b_v")
     outs = []
     for b in range(B):
         cache = {}
-        for n in ("a_k", "a_v", "b_k", "b_v"):
+        for n in cached:
             head = prior[n][b][:start_pos] if (prior is not None and start_pos) else \
                 np.zeros((0,) + new[n].shape[2:])
             cache[n] = np.concatenate([np.asarray(head, np.float64), new[n][b]], axis=0)
+        if dims.shared_basis:
+            cache.update(broadcast_basis(basis, cache["a_k"].shape[0], dims))
         if dims.rank_q == 0:
             q = new["q"][b]                               # TPA-KVonly: plain query
         else:
@@ -314,17 +353,20 @@ def output_projection(out: np.ndarray, w_o: np.ndarray) -> np.ndarray:
 
 
 def tpa_forward_rows(x: np.ndarray, w_cat: np.ndarray, dims: Dims, rope_base: float,
-                     rows) -> np.ndarray:
+                     rows, basis: dict | None = None) -> np.ndarray:
     """``tpa_forward`` for one sequence that starts at position 0, evaluated only for
     the query rows ``rows`` (the keys and values still cover the whole sequence), so
     that long sequences can be checked on a sample of their outputs.
 
     x: [S, d_model].  Returns out [len(rows), h, d].  Same steps, same order as
-    ``tpa_forward``: project, materialise, rotate the materialised q and k, attend.
+    ``tpa_forward``: project, materialise, rotate the materialised q and k, attend
+    (``basis`` as in ``tpa_forward``).
     """
     x = np.asarray(x, dtype=np.float64)
     rows = np.asarray(rows).reshape(-1)
     f = project(x, w_cat, dims)
+    if dims.shared_basis:
+        f.update(broadcast_basis(basis, x.shape[0], dims))
     if dims.rank_q == 0:
         q = f["q"][rows]                                  # TPA-KVonly: plain query
     else:

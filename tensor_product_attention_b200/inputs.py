@@ -23,7 +23,8 @@ import torch
 
 # stream tags, so that each tensor of a workload has its own random stream
 _TAG = {"x": 1, "w": 2, "len": 3, "a_k": 4, "a_v": 5, "b_k": 6, "b_v": 7,
-        "a_q": 8, "b_q": 9, "q": 10, "misc": 11, "wo": 12, "o": 13}
+        "a_q": 8, "b_q": 9, "q": 10, "misc": 11, "wo": 12, "o": 13,
+        "basis_k": 14, "basis_v": 15}
 
 
 @dataclass(frozen=True)
@@ -44,10 +45,12 @@ class Workload:
     seqlen: int = 0      # prefill: tokens per sequence
     d_model: int = 0     # prefill: model width
     context: tuple = field(default=(0, 0))   # decode: (min, max) context length
+    shared_basis: bool = False   # B_K, B_V are layer parameters shared by all tokens
 
     def dims(self):
         return dict(d_model=self.d_model, n_heads=self.n_heads, head_dim=self.head_dim,
-                    rank_q=self.rank_q, rank_k=self.rank_k, rank_v=self.rank_v)
+                    rank_q=self.rank_q, rank_k=self.rank_k, rank_v=self.rank_v,
+                    shared_basis=self.shared_basis)
 
 
 WORKLOADS = {
@@ -72,6 +75,11 @@ WORKLOADS = {
         Workload("kvonly_layer_prefill_b4_s8192_d4096", "prefill", "bf16", batch=4, seqlen=8192,
                  d_model=4096, n_heads=32, head_dim=128, rank_q=0, rank_k=2, rank_v=2,
                  rope_base=5e5, seed=1006),
+        # shared-basis variant (B_K, B_V shared across tokens): the decode shape of
+        # decode_b64_ctx32k with only A_K, A_V cached per token
+        Workload("shared_basis_decode_b64_ctx32k", "decode", "bf16", batch=64,
+                 context=(32768, 32768), n_heads=16, head_dim=128, rank_q=6, rank_k=2,
+                 rank_v=2, rope_base=1e4, seed=1007, shared_basis=True),
     )
 }
 
@@ -101,12 +109,14 @@ def torch_dtype(dtype: str):
     return {"bf16": torch.bfloat16, "f32": torch.float32}[dtype]
 
 
-def factor_widths(n_heads, head_dim, rank_q, rank_k, rank_v):
+def factor_widths(n_heads, head_dim, rank_q, rank_k, rank_v, shared_basis=False):
     """Rows of the stacked projection weight: W_A_q, W_A_k, W_A_v, W_B_q, W_B_k, W_B_v.
     TPA-KVonly (rank_q = 0): no W_A_q rows, and the W_B_q block is the plain query
-    projection with n_heads * head_dim rows."""
+    projection with n_heads * head_dim rows.  Shared basis: no W_B_k, W_B_v rows."""
+    kb = 0 if shared_basis else rank_k * head_dim
+    vb = 0 if shared_basis else rank_v * head_dim
     return [n_heads * rank_q, n_heads * rank_k, n_heads * rank_v,
-            (rank_q if rank_q > 0 else n_heads) * head_dim, rank_k * head_dim, rank_v * head_dim]
+            (rank_q if rank_q > 0 else n_heads) * head_dim, kb, vb]
 
 
 # ------------------------------------------------------------------- prefill inputs
@@ -119,7 +129,7 @@ def prefill_x(wl: Workload, b: int, seqlen: int | None = None, seed: int | None 
 
 def prefill_w(wl: Workload, seed: int | None = None) -> torch.Tensor:
     """The six stacked projection weights: [sum of widths, d_model] ~ N(0, 1/d_model)."""
-    n = sum(factor_widths(wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v))
+    n = sum(factor_widths(wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v, wl.shared_basis))
     g = rng(wl.seed if seed is None else seed, "w")
     return to_storage(normal(g, (n, wl.d_model), 1.0 / np.sqrt(wl.d_model)), wl.dtype)
 
@@ -137,6 +147,15 @@ def attn_out(wl: Workload, T: int, seed: int | None = None) -> torch.Tensor:
     return to_storage(normal(g, (T, wl.n_heads, wl.head_dim), 1.0 / np.sqrt(wl.head_dim)), wl.dtype)
 
 
+def shared_basis(wl: Workload, seed: int | None = None) -> dict:
+    """The layer's shared key and value basis (shared-basis variant), un-rotated:
+    b_k [R_K, d_h], b_v [R_V, d_h] ~ N(0, 1/d_h), like the per-token B factors."""
+    s = wl.seed if seed is None else seed
+    sd = 1.0 / np.sqrt(wl.head_dim)
+    return {"b_k": to_storage(normal(rng(s, "basis_k"), (wl.rank_k, wl.head_dim), sd), wl.dtype),
+            "b_v": to_storage(normal(rng(s, "basis_v"), (wl.rank_v, wl.head_dim), sd), wl.dtype)}
+
+
 # -------------------------------------------------------------------- decode inputs
 
 def decode_lengths(wl: Workload) -> np.ndarray:
@@ -152,16 +171,18 @@ def decode_sequence(wl: Workload, b: int, length: int, a_scale: float = 1.0) -> 
     a_k, a_v: [length, h, R] ~ N(0, a_scale^2); b_k, b_v: [length, R, d] ~ N(0, 1/d);
     query a_q: [h, R_Q] ~ N(0, a_scale^2) and b_q: [R_Q, d] ~ N(0, 1/d), or, for
     TPA-KVonly, q: [h, d] ~ N(0, 1/d).  ``a_scale`` > 1 sharpens the softmax (the
-    configured scales give a nearly uniform one).
+    configured scales give a nearly uniform one).  Shared-basis workloads have no
+    per-token b_k, b_v (see ``shared_basis``).
     """
     h, d, s = wl.n_heads, wl.head_dim, wl.seed
     sd = 1.0 / np.sqrt(d)
     out = {
         "a_k": to_storage(normal(rng(s, "a_k", b), (length, h, wl.rank_k), a_scale), wl.dtype),
         "a_v": to_storage(normal(rng(s, "a_v", b), (length, h, wl.rank_v), a_scale), wl.dtype),
-        "b_k": to_storage(normal(rng(s, "b_k", b), (length, wl.rank_k, d), sd), wl.dtype),
-        "b_v": to_storage(normal(rng(s, "b_v", b), (length, wl.rank_v, d), sd), wl.dtype),
     }
+    if not wl.shared_basis:
+        out["b_k"] = to_storage(normal(rng(s, "b_k", b), (length, wl.rank_k, d), sd), wl.dtype)
+        out["b_v"] = to_storage(normal(rng(s, "b_v", b), (length, wl.rank_v, d), sd), wl.dtype)
     if wl.rank_q == 0:
         out["q"] = to_storage(normal(rng(s, "q", b), (h, d), sd), wl.dtype)
     else:
@@ -174,15 +195,17 @@ def prefill_factors(wl: Workload, b: int, n_query: int, n_keys: int, a_scale: fl
     """Factors for attention-only prefill checks of sequence ``b``: cached K/V factors
     for ``n_keys`` tokens (B_K already rotated) and query factors for ``n_query``
     tokens (B_Q already rotated), same distributions as ``decode_sequence``; for
-    TPA-KVonly the query is ``q`` [n_query, h, d] ~ N(0, 1/d)."""
+    TPA-KVonly the query is ``q`` [n_query, h, d] ~ N(0, 1/d).  Shared-basis workloads
+    have no per-token b_k, b_v."""
     h, d, s = wl.n_heads, wl.head_dim, wl.seed
     sd = 1.0 / np.sqrt(d)
     out = {
         "a_k": to_storage(normal(rng(s, "a_k", b), (n_keys, h, wl.rank_k), a_scale), wl.dtype),
         "a_v": to_storage(normal(rng(s, "a_v", b), (n_keys, h, wl.rank_v), a_scale), wl.dtype),
-        "b_k": to_storage(normal(rng(s, "b_k", b), (n_keys, wl.rank_k, d), sd), wl.dtype),
-        "b_v": to_storage(normal(rng(s, "b_v", b), (n_keys, wl.rank_v, d), sd), wl.dtype),
     }
+    if not wl.shared_basis:
+        out["b_k"] = to_storage(normal(rng(s, "b_k", b), (n_keys, wl.rank_k, d), sd), wl.dtype)
+        out["b_v"] = to_storage(normal(rng(s, "b_v", b), (n_keys, wl.rank_v, d), sd), wl.dtype)
     if wl.rank_q == 0:
         out["q"] = to_storage(normal(rng(s, "q", b), (n_query, h, d), sd), wl.dtype)
     else:

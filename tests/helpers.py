@@ -31,10 +31,11 @@ def dims_of(wl, binding):
 def fill_cache(cache, b, seq: dict, start: int = 0):
     """Copy one sequence's seeded factors into cache slot b at [start, start+L) (plumbing)."""
     n = seq["a_k"].shape[0]
-    for name in ("a_k", "a_v", "b_k", "b_v"):
+    for name in ("a_k", "a_v") if "b_k" not in seq else ("a_k", "a_v", "b_k", "b_v"):
         getattr(cache, name)[b, start:start + n].copy_(seq[name], non_blocking=False)
 
 
 def oracle_dims(wl):
     import oracle
-    return oracle.Dims(wl.d_model, wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v)
+    return oracle.Dims(wl.d_model, wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v,
+                       shared_basis=wl.shared_basis)

@@ -476,3 +476,138 @@ def test_output_projection_is_a_bias_free_linear_on_flattened_heads():
     # head-major flattening: feature h*d + k of the input is head h, dim k
     e = np.zeros((1, h, d)); e[0, 2, 1] = 1.0
     assert rel(oracle.output_projection(e, w_o)[0], w_o[:, 2 * d + 1]) < TOL
+
+
+# ------------------------------------------------------- shared-basis variant
+
+def _shared_case(g, dims, B, S):
+    widths = oracle.factor_widths(dims)
+    assert widths["b_k"] == 0 and widths["b_v"] == 0
+    ws = {n: g.standard_normal((widths[n], dims.d_model)) / math.sqrt(dims.d_model) for n in oracle.FACTOR_NAMES}
+    basis = {"b_k": g.standard_normal((dims.rank_k, dims.head_dim)),
+             "b_v": g.standard_normal((dims.rank_v, dims.head_dim))}
+    x = g.standard_normal((B, S, dims.d_model))
+    return ws, np.concatenate([ws[n] for n in oracle.FACTOR_NAMES], axis=0), basis, x
+
+
+def _torch_rope(t, positions, base):
+    """RoPE as complex multiplication of interleaved pairs; t [S, n, d] (fp64 torch)."""
+    S, n, d = t.shape
+    theta = torch.tensor(base, dtype=torch.float64) ** (-(torch.arange(0, d, 2, dtype=torch.float64) / d))
+    pos = torch.as_tensor(np.asarray(positions), dtype=torch.float64)
+    rot = torch.polar(torch.ones(S, d // 2, dtype=torch.float64), pos[:, None] * theta[None, :])
+    c = torch.view_as_complex(t.reshape(S, n, d // 2, 2).contiguous())
+    return torch.view_as_real(c * rot[:, None, :]).reshape(S, n, d)
+
+
+def test_shared_basis_projection_has_no_per_token_key_value_basis():
+    # [review] 优点与创新 5: basis vectors shared across tokens.  Reading: W_B_k and
+    # W_B_v are gone; the cache keeps (R_K + R_V) h elements per token.
+    g = gen(31)
+    dims = Dims(d_model=24, n_heads=3, head_dim=8, rank_q=2, rank_k=2, rank_v=3, shared_basis=True)
+    ws, w_cat, _, x = _shared_case(g, dims, 1, 5)
+    assert w_cat.shape[0] == 3 * (2 + 2 + 3) + 2 * 8
+    got = oracle.project(x[0], w_cat, dims)
+    assert set(got) == {"a_q", "b_q", "a_k", "a_v"}
+    want_av = F.linear(torch.from_numpy(x[0]), torch.from_numpy(ws["a_v"])).view(5, 3, 3).numpy()
+    assert rel(got["a_v"], want_av) < TOL
+    assert oracle.cache_elements_per_token(dims) == (2 + 3) * 3
+    # same layer with a contextual basis: the per-token B side is what the variant drops
+    ctx = Dims(24, 3, 8, 2, 2, 3)
+    assert oracle.cache_elements_per_token(ctx) - oracle.cache_elements_per_token(dims) == (2 + 3) * 8
+
+
+def test_shared_basis_forward_is_textbook_attention_on_materialised_kv():
+    # Independent route in torch: F.linear for the A projections and the query, K and V
+    # as (1/R) a . basis with matmul, RoPE as complex multiplication on q and k,
+    # causal fp64 scaled_dot_product_attention.
+    g = gen(32)
+    dims = Dims(d_model=20, n_heads=4, head_dim=8, rank_q=3, rank_k=2, rank_v=3, shared_basis=True)
+    B, S, base = 2, 13, 1e4
+    ws, w_cat, basis, x = _shared_case(g, dims, B, S)
+    out, new = oracle.tpa_forward(x, w_cat, dims, base, basis=basis)
+    h, d = dims.n_heads, dims.head_dim
+    bk, bv = torch.from_numpy(basis["b_k"]), torch.from_numpy(basis["b_v"])
+    tables = oracle.shared_basis_tables(basis, dims, S + 3, base)
+    for b in range(B):
+        xt = torch.from_numpy(x[b])
+        lin = {n: F.linear(xt, torch.from_numpy(ws[n])) for n in oracle.FACTOR_NAMES if ws[n].shape[0]}
+        q = torch.bmm(lin["a_q"].view(S, h, 3), lin["b_q"].view(S, 3, d)) / 3
+        k = torch.matmul(lin["a_k"].view(S, h, 2), bk) / 2
+        v = torch.matmul(lin["a_v"].view(S, h, 3), bv) / 3
+        q, k = _torch_rope(q, np.arange(S), base), _torch_rope(k, np.arange(S), base)
+        want = F.scaled_dot_product_attention(q.permute(1, 0, 2), k.permute(1, 0, 2), v.permute(1, 0, 2),
+                                              is_causal=True).permute(1, 0, 2)
+        assert rel(out[b], want.numpy()) < 1e-12
+        # the pre-rotated form the kernels use: query factors rotated at their positions,
+        # keys read against the per-position tables (row j = basis rotated at j)
+        qf = {"a_q": new["a_q"][b], "b_q": oracle.rope_rotate(new["b_q"][b], np.arange(S), base)}
+        kv = {"a_k": new["a_k"][b], "a_v": new["a_v"][b],
+              "b_k": tables["b_k"][:S], "b_v": tables["b_v"][:S]}
+        assert rel(oracle.attend_from_factors(qf, kv, dims, np.arange(S)), out[b]) < 1e-12
+        dec = oracle.decode_attention({"a_q": qf["a_q"][S - 1], "b_q": qf["b_q"][S - 1]}, kv, dims, S)
+        assert rel(dec, out[b, S - 1]) < 1e-12
+    rows = [0, 7, 12]
+    assert rel(oracle.tpa_forward_rows(x[1], w_cat, dims, base, rows, basis=basis), out[1, rows]) < 1e-12
+    # a second chunk after a cached prefix gives the rows of the one-shot pass
+    head, new_h = oracle.tpa_forward(x[:, :8], w_cat, dims, base, basis=basis)
+    tail, _ = oracle.tpa_forward(x[:, 8:], w_cat, dims, base, start_pos=8, prior=new_h, basis=basis)
+    assert rel(np.concatenate([head, tail], axis=1), out) < 1e-12
+
+
+def test_shared_basis_with_identity_basis_is_mha():
+    # With R_K = R_V = d_h and the identity as the shared basis, the key of head h is
+    # its own contextual d_h-vector a^K_{t,h,:} / d_h: plain MHA with key and value
+    # projections W_A_k / R_K and W_A_v / R_V (the per-head view of 类定义与初始化).
+    g = gen(33)
+    h, d, D, S, base = 3, 8, 16, 9, 1e4
+    dims = Dims(d_model=D, n_heads=h, head_dim=d, rank_q=0, rank_k=d, rank_v=d, shared_basis=True)
+    ws, w_cat, _, x = _shared_case(g, dims, 1, S)
+    basis = {"b_k": np.eye(d), "b_v": np.eye(d)}
+    out, _ = oracle.tpa_forward(x, w_cat, dims, base, basis=basis)
+    xt = torch.from_numpy(x[0])
+    q = F.linear(xt, torch.from_numpy(ws["b_q"])).view(S, h, d)
+    k = F.linear(xt, torch.from_numpy(ws["a_k"] / d)).view(S, h, d)
+    v = F.linear(xt, torch.from_numpy(ws["a_v"] / d)).view(S, h, d)
+    q, k = _torch_rope(q, np.arange(S), base), _torch_rope(k, np.arange(S), base)
+    want = F.scaled_dot_product_attention(q.permute(1, 0, 2), k.permute(1, 0, 2), v.permute(1, 0, 2),
+                                          is_causal=True).permute(1, 0, 2)
+    assert rel(out[0], want.numpy()) < 1e-12
+
+
+def test_shared_basis_tables_closed_form():
+    # Row p of the key table is the basis turned by p * theta_k per pair; for the unit
+    # vector e_0 (theta_0 = 1) that is (cos p, sin p, 0, ...).  The value table is the
+    # basis itself on every row.
+    dims = Dims(0, 1, 4, 0, 2, 1, shared_basis=True)
+    e = np.zeros((2, 4)); e[0, 0] = 1.0; e[1, 3] = 1.0
+    bv = np.array([[0.5, -1.0, 2.0, 0.25]])
+    t = oracle.shared_basis_tables({"b_k": e, "b_v": bv}, dims, 5, 100.0)
+    assert t["b_k"].shape == (5, 2, 4) and t["b_v"].shape == (5, 1, 4)
+    for p in range(5):
+        np.testing.assert_allclose(t["b_k"][p, 0], [math.cos(p), math.sin(p), 0, 0], atol=TOL)
+        a = p * 100.0 ** (-2 / 4)                  # pair 1 turns by p * base^(-1/2)
+        np.testing.assert_allclose(t["b_k"][p, 1], [0, 0, -math.sin(a), math.cos(a)], atol=TOL)
+        np.testing.assert_array_equal(t["b_v"][p], bv)
+
+
+def test_shared_basis_planted_mistakes_are_caught(monkeypatch):
+    real = oracle.tpa_oracle.shared_basis_tables
+    real_bb = oracle.tpa_oracle.broadcast_basis
+
+    # 1. tables rotated one position late
+    def late(basis, dims, capacity, base):
+        t = real(basis, dims, capacity + 1, base)
+        return {"b_k": t["b_k"][1:], "b_v": t["b_v"][1:]}
+    assert _pins_fail(monkeypatch, "shared_basis_tables", late,
+                      [test_shared_basis_tables_closed_form,
+                       test_shared_basis_forward_is_textbook_attention_on_materialised_kv]) == 2
+    monkeypatch.setattr(oracle.tpa_oracle, "shared_basis_tables", real)
+    monkeypatch.setattr(oracle, "shared_basis_tables", real)
+
+    # 2. the basis vectors read back to front along d_h
+    def reversed_d(basis, n_tokens, dims):
+        out = real_bb(basis, n_tokens, dims)
+        return {n: np.ascontiguousarray(t[..., ::-1]) for n, t in out.items()}
+    assert _pins_fail(monkeypatch, "broadcast_basis", reversed_d,
+                      [test_shared_basis_forward_is_textbook_attention_on_materialised_kv]) == 1
