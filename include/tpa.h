@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define TPA_ABI_VERSION 1
+#define TPA_ABI_VERSION 2
 #define TPA_MAX_BATCH 1024          /* sequences per call */
 
 typedef struct CUstream_st* tpa_stream_t;   /* same type as cudaStream_t */
@@ -71,7 +71,12 @@ typedef enum tpa_dtype { TPA_F32 = 0, TPA_BF16 = 1 } tpa_dtype;
 /* Shape of one TPA layer: the page's ModelArgs (dim, n_heads, head_dim, q_rank, rank)
  * [review, 代码 类定义与初始化], with rank split into rank_k and rank_v.
  * rank_q = 0 selects TPA-KVonly [review, 实验/结果]: the query is a plain per-head
- * vector [h][d_h] held in the b_q slot; a_q is unused. */
+ * vector [h][d_h] held in the b_q slot; a_q is unused.
+ * shared_basis = 1 selects the variant that shares the basis vectors across tokens
+ * [review, 优点与创新 5], named there in one clause.  Reading taken: B_K and B_V are
+ * layer parameters (basis_k [R_K][d_h], basis_v [R_V][d_h]), the same for every
+ * token; A_K, A_V and the query stay contextual; RoPE turns the key at its position.
+ * Only A_K and A_V are cached per token.  The per-call effects are stated below. */
 typedef struct tpa_dims {
     int32_t d_model;
     int32_t n_heads;     /* h */
@@ -80,6 +85,7 @@ typedef struct tpa_dims {
     int32_t rank_k;      /* R_K */
     int32_t rank_v;      /* R_V */
     int32_t dtype;       /* tpa_dtype */
+    int32_t shared_basis;  /* 0: contextual B_K, B_V (TPA); 1: shared basis */
 } tpa_dims;
 
 /* The six factor tensors of T tokens (device):
@@ -95,7 +101,9 @@ typedef struct tpa_factors {
 /* The factor cache of `batch` sequences with room for `capacity` tokens each (device),
  * the page's cache_kA / cache_vA / cache_kB / cache_vB [review, 类定义与初始化]:
  *   a_k, a_v [batch][capacity][h][R]    b_k, b_v [batch][capacity][R][d_h]
- * lengths [batch] int32 (device) is written by tpa_cache_append. */
+ * lengths [batch] int32 (device) is written by tpa_cache_append.
+ * Shared basis (dims->shared_basis = 1): b_k and b_v are the layer's per-position
+ * tables [capacity][R][d_h] from tpa_shared_basis_tables, read by every sequence. */
 typedef struct tpa_cache {
     void* a_k; void* a_v;
     void* b_k; void* b_v;
@@ -110,7 +118,8 @@ const char* tpa_build_info(void);
 const char* tpa_status_string(tpa_status status);
 
 /* Bytes the factor cache holds per token: (R_K + R_V) * (h + d_h) * sizeof(element),
- * from the page's cache shapes [review, 类定义与初始化].  0 for invalid dims. */
+ * from the page's cache shapes [review, 类定义与初始化]; (R_K + R_V) * h * sizeof(element)
+ * with a shared basis (the per-layer tables are not per token).  0 for invalid dims. */
 size_t tpa_cache_bytes_per_token(const tpa_dims* dims);
 
 /* RoPE table: cs[p][k][0] = cos(p * theta_k), cs[p][k][1] = sin(p * theta_k) for
@@ -134,7 +143,9 @@ tpa_status tpa_rope_table(const tpa_dims* dims, double base, int32_t max_pos,
  * query projection W_Q with h*d_h rows (row h*d_h + k is head h, dim k), so N =
  * h(R_K+R_V) + d_h(h+R_K+R_V); out->b_q receives the rotated query [T][h][d_h] and
  * out->a_q may be NULL.  The pages do not print this variant's projection; this
- * layout is the reading taken. */
+ * layout is the reading taken.
+ * Shared basis: the W_B_k and W_B_v blocks are absent (N = h(R_Q+R_K+R_V) + d_h R_Q,
+ * or the KV-only count without them) and out->b_k, out->b_v are not used (may be NULL). */
 tpa_status tpa_project(const tpa_dims* dims, const void* x, const void* w_cat,
                        int32_t batch, int32_t seqlen, const int32_t* start_pos,
                        const float* rope_cs, int32_t max_pos,
@@ -146,10 +157,27 @@ tpa_status tpa_project(const tpa_dims* dims, const void* x, const void* w_cat,
  * cache[:bsz, start_pos:start_pos+seqlen] = factors [review, 代码 前向传播].
  *   kv         device factors for batch*n_tokens tokens (a_q, b_q ignored)
  *   start_pos  host [batch]; start_pos[b] + n_tokens <= capacity (else TPA_ERR_CAPACITY)
- * batch <= cache->batch; sequences >= batch are left alone. */
+ * batch <= cache->batch; sequences >= batch are left alone.
+ * Shared basis: only a_k and a_v are copied; kv->b_k, kv->b_v may be NULL. */
 tpa_status tpa_cache_append(const tpa_dims* dims, const tpa_cache* cache,
                             const tpa_factors* kv, int32_t batch, int32_t n_tokens,
                             const int32_t* start_pos, tpa_stream_t stream);
+
+/* Shared-basis tables (dims->shared_basis = 1) for a cache of `capacity` positions:
+ *   table_k[p][s][:] = basis_k[s] rotated at position p (RoPE as tpa_project rotates
+ *                      B_K: fp32 arithmetic, rounded once to dims->dtype)
+ *   table_v[p][s][:] = basis_v[s]
+ * This is the cache side of the shared basis, pre-rotated as B_K is cached [review,
+ * 问题2]: one table per layer, not per sequence.  Set cache->b_k = table_k and
+ * cache->b_v = table_v.  Rebuild after changing the basis.
+ *   basis_k  device [R_K][d_h]      basis_v device [R_V][d_h]
+ *   rope_cs  device table from tpa_rope_table with max_pos >= capacity rows
+ *   table_k  device [capacity][R_K][d_h]   table_v device [capacity][R_V][d_h]
+ * TPA_ERR_INVALID if dims->shared_basis is 0; TPA_ERR_CAPACITY if capacity > max_pos. */
+tpa_status tpa_shared_basis_tables(const tpa_dims* dims, const void* basis_k,
+                                   const void* basis_v, const float* rope_cs,
+                                   int32_t max_pos, int32_t capacity, void* table_k,
+                                   void* table_v, tpa_stream_t stream);
 
 /* Causal prefill from factors: query i of sequence b (position p = start_pos[b] + i)
  * attends to cached keys 0..p of sequence b:
@@ -160,7 +188,8 @@ tpa_status tpa_cache_append(const tpa_dims* dims, const tpa_cache* cache,
  *          TPA-KVonly: b_q = the rotated query [T][h][d_h], a_q ignored
  *   cache  must already hold positions 0 .. start_pos[b]+seqlen-1 of each sequence
  *   start_pos host [batch]
- *   out    device [batch*seqlen][h][d_h] */
+ *   out    device [batch*seqlen][h][d_h]
+ * Shared basis: key j of every sequence reads row j of cache->b_k and cache->b_v. */
 tpa_status tpa_prefill(const tpa_dims* dims, const tpa_factors* q, const tpa_cache* cache,
                        int32_t batch, int32_t seqlen, const int32_t* start_pos,
                        void* out, tpa_stream_t stream);
@@ -177,7 +206,9 @@ tpa_status tpa_prefill(const tpa_dims* dims, const tpa_factors* q, const tpa_cac
  *   lengths  host [batch], 1 <= lengths[b] <= capacity
  *   out      device [batch][h][d_h]
  *   workspace device scratch of at least tpa_decode_workspace_bytes() bytes, 256-byte
- *            aligned; contents on entry do not matter and are undefined on return. */
+ *            aligned; contents on entry do not matter and are undefined on return.
+ * Shared basis: keys read A_K, A_V from the sequence's cache rows and B_K, B_V from
+ * the per-position tables (so per key only (R_K + R_V) h elements come from HBM). */
 tpa_status tpa_decode(const tpa_dims* dims, const void* q_a, const void* q_b,
                       const tpa_cache* cache, const int32_t* lengths, int32_t batch,
                       void* out, void* workspace, size_t workspace_bytes,
@@ -204,7 +235,8 @@ size_t tpa_decode_workspace_bytes(const tpa_dims* dims, const int32_t* lengths, 
  *   workspace device scratch of at least tpa_decode_step_workspace_bytes() bytes,
  *            256-byte aligned: the new tokens' query factors, then decode's partials.
  * Arguments are checked before anything is launched (TPA_ERR_CAPACITY when a
- * sequence has no room or its position is past the RoPE table). */
+ * sequence has no room or its position is past the RoPE table).
+ * Shared basis: only A_K, A_V are written into the cache (w_cat without W_B_k, W_B_v). */
 tpa_status tpa_decode_step(const tpa_dims* dims, const void* x, const void* w_cat,
                            const float* rope_cs, int32_t max_pos, const tpa_cache* cache,
                            const int32_t* lengths, int32_t batch, void* out,

@@ -28,15 +28,16 @@ TPA_MAX_BATCH = 1024
 EXPORTS = ("tpa_abi_version", "tpa_build_info", "tpa_status_string", "tpa_cache_bytes_per_token",
            "tpa_rope_table", "tpa_project", "tpa_cache_append", "tpa_prefill", "tpa_decode",
            "tpa_decode_workspace_bytes", "tpa_decode_static", "tpa_decode_step",
-           "tpa_decode_step_workspace_bytes", "tpa_output_project", "tpa_get_device_error",
-           "tpa_set_wait_limit")
+           "tpa_decode_step_workspace_bytes", "tpa_output_project", "tpa_shared_basis_tables",
+           "tpa_get_device_error", "tpa_set_wait_limit")
 TPA_DECODE_STATIC_SCRATCH_BYTES = 16 << 20
 
 
 class tpa_dims(ctypes.Structure):
     _fields_ = [("d_model", ctypes.c_int32), ("n_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("rank_q", ctypes.c_int32),
-                ("rank_k", ctypes.c_int32), ("rank_v", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+                ("rank_k", ctypes.c_int32), ("rank_v", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("shared_basis", ctypes.c_int32)]
 
 
 class tpa_factors(ctypes.Structure):
@@ -77,6 +78,9 @@ _sig = {
     "tpa_decode_step_workspace_bytes": (ctypes.c_size_t, [_P(tpa_dims), _i32p, ctypes.c_int32]),
     "tpa_output_project": (ctypes.c_int, [_P(tpa_dims), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
                                           ctypes.c_void_p, ctypes.c_void_p]),
+    "tpa_shared_basis_tables": (ctypes.c_int, [_P(tpa_dims), ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "tpa_get_device_error": (ctypes.c_int, [ctypes.c_void_p, _i32p]),
     "tpa_set_wait_limit": (None, [ctypes.c_uint32]),
 }
@@ -109,10 +113,11 @@ class Dims:
     rank_k: int
     rank_v: int
     dtype: int = BF16
+    shared_basis: int = 0      # 1: B_K, B_V shared across tokens (per-position tables)
 
     def c(self) -> tpa_dims:
         return tpa_dims(self.d_model, self.n_heads, self.head_dim, self.rank_q, self.rank_k,
-                        self.rank_v, self.dtype)
+                        self.rank_v, self.dtype, int(self.shared_basis))
 
     @property
     def torch_dtype(self):
@@ -120,8 +125,11 @@ class Dims:
 
     @property
     def n_proj(self) -> int:
-        r = self.rank_q + self.rank_k + self.rank_v
-        return r * (self.n_heads + self.head_dim)
+        """Rows of the stacked projection weight w_cat (tpa_project)."""
+        h, d = self.n_heads, self.head_dim
+        q_rows = self.rank_q if self.rank_q > 0 else h
+        kv_b = 0 if self.shared_basis else (self.rank_k + self.rank_v) * d
+        return h * (self.rank_q + self.rank_k + self.rank_v) + q_rows * d + kv_b
 
 
 @dataclass
@@ -172,18 +180,22 @@ def alloc_factors(dims: Dims, T: int, device="cuda", queries=True, kv=True) -> F
         f.b_q = torch.empty((T, h, d), dtype=dt, device=device)
     if kv:
         f.a_k = torch.empty((T, h, dims.rank_k), dtype=dt, device=device)
-        f.b_k = torch.empty((T, dims.rank_k, d), dtype=dt, device=device)
         f.a_v = torch.empty((T, h, dims.rank_v), dtype=dt, device=device)
-        f.b_v = torch.empty((T, dims.rank_v, d), dtype=dt, device=device)
+        if not dims.shared_basis:
+            f.b_k = torch.empty((T, dims.rank_k, d), dtype=dt, device=device)
+            f.b_v = torch.empty((T, dims.rank_v, d), dtype=dt, device=device)
     return f
 
 
 def alloc_cache(dims: Dims, batch: int, capacity: int, device="cuda", fill=None) -> Cache:
+    """Cache tensors; with a shared basis b_k, b_v are the per-position tables
+    [capacity][R][d_h] (fill them with tpa_shared_basis_tables)."""
     h, d, dt = dims.n_heads, dims.head_dim, dims.torch_dtype
     mk = (lambda s: torch.full(s, fill, dtype=dt, device=device)) if fill is not None else \
         (lambda s: torch.empty(s, dtype=dt, device=device))
+    lead = (capacity,) if dims.shared_basis else (batch, capacity)
     return Cache(mk((batch, capacity, h, dims.rank_k)), mk((batch, capacity, h, dims.rank_v)),
-                 mk((batch, capacity, dims.rank_k, d)), mk((batch, capacity, dims.rank_v, d)),
+                 mk(lead + (dims.rank_k, d)), mk(lead + (dims.rank_v, d)),
                  torch.zeros(batch, dtype=torch.int32, device=device))
 
 
@@ -233,6 +245,15 @@ def tpa_cache_append(dims: Dims, cache: Cache, kv: Factors, batch: int, n_tokens
     _check("tpa_cache_append", _lib.tpa_cache_append(ctypes.byref(dims.c()), ctypes.byref(cache.c()),
                                                      ctypes.byref(kv.c()), int(batch), int(n_tokens),
                                                      _ints(start_pos), _stream(stream)))
+
+
+def tpa_shared_basis_tables(dims: Dims, basis_k, basis_v, rope_cs, max_pos: int, table_k, table_v,
+                            stream=None) -> None:
+    """Shared basis: table_k[p] = basis_k rotated at position p, table_v[p] = basis_v,
+    for p < table_k.shape[0] (the cache capacity)."""
+    _check("tpa_shared_basis_tables", _lib.tpa_shared_basis_tables(
+        ctypes.byref(dims.c()), _ptr(basis_k), _ptr(basis_v), _ptr(rope_cs), int(max_pos),
+        int(table_k.shape[0]), _ptr(table_k), _ptr(table_v), _stream(stream)))
 
 
 def tpa_prefill(dims: Dims, q: Factors, cache: Cache, batch: int, seqlen: int, start_pos, out,

@@ -97,6 +97,7 @@ struct DecodeArgs {
     float* ws_ml;   // [parts][H][2]
     float* ws_o;    // [parts][H][Dh]
     int H, Dh, Rq, Rk, Rv, cap, split_len;
+    long long bcap;   // B_K / B_V rows between sequences: cap, or 0 (shared basis)
 };
 
 template <typename T>
@@ -146,17 +147,17 @@ __global__ void __launch_bounds__(NT) decode_simt_kernel(DecodeArgs a, const Dec
     const T* av = reinterpret_cast<const T*>(a.ca_v);
     const T* bk = reinterpret_cast<const T*>(a.cb_k);
     const T* bv = reinterpret_cast<const T*>(a.cb_v);
-    const long long seq_row = (long long)b * a.cap;
+    const long long seq_row = (long long)b * a.cap, bseq_row = (long long)b * a.bcap;
 
     for (int jt = j0; jt < j1; jt += KT) {
         const int n = min(KT, j1 - jt);
         __syncthreads();
         for (int u = tid; u < n * a.Rk * Dh; u += NT) {
             int j = u / (a.Rk * Dh), r = u - j * (a.Rk * Dh);
-            bks[j * bk_row + r] = to_f(bk[(seq_row + jt) * a.Rk * Dh + u]);
+            bks[j * bk_row + r] = to_f(bk[(bseq_row + jt) * a.Rk * Dh + u]);
         }
         for (int u = tid; u < n * a.Rv * Dh; u += NT)
-            bvs[u] = to_f(bv[(seq_row + jt) * a.Rv * Dh + u]);
+            bvs[u] = to_f(bv[(bseq_row + jt) * a.Rv * Dh + u]);
         for (int u = tid; u < n * H * a.Rk; u += NT) {
             int j = u / (H * a.Rk), hr = u - j * (H * a.Rk);
             akT[hr * KT + j] = to_f(ak[(seq_row + jt) * H * a.Rk + u]);
@@ -279,6 +280,7 @@ cudaError_t launch_decode_simt(const Shape& s, const void* q_a, const void* q_b,
     a.ws_ml = ws;
     a.ws_o = ws + (size_t)plan.total_parts * s.H * 2;
     a.H = s.H; a.Dh = s.Dh; a.Rq = s.Rq; a.Rk = s.Rk; a.Rv = s.Rv; a.cap = c.capacity;
+    a.bcap = b_seq_rows(s, c);
     a.split_len = plan.split_len;
     size_t smem = decode_simt_smem(s);
     if (smem > 227 * 1024) return cudaErrorInvalidValue;

@@ -23,6 +23,12 @@
 // Warp roles: warp 0 TMA (two stages of b^K/b^V tiles, 128-byte swizzle, and a^K/a^V
 // bulk copies), warp 1 TMEM owner and MMA issuer, warps 2.. softmax (4 warps per 16
 // heads; TMEM lane = row).  TMEM: U^T double-buffered (2 x h columns) and O^T (h).
+//
+// Shared basis (B_K, B_V shared across tokens, same page, 优点与创新 5): b^K tiles come
+// from the layer's per-position table (row j = the key basis rotated at j, the same for
+// every sequence, so it is read through L2), and every b^V row of a tile is the value
+// basis, so one V stage is loaded once and reused by every PV.  Per key only the
+// (R_K + R_V) h A factors come from the sequence's cache.
 #include <algorithm>
 #include <cmath>
 
@@ -47,6 +53,7 @@ struct DecodeTcArgs {
     float* ws_ml;                  // [parts][H][2]
     float* ws_o;                   // [parts][H][DH]
     int Rq, cap;
+    int bcap;                      // B rows between sequences: cap, or 0 (shared basis)
     int asw;                       // a^K, a^V tiles by TMA with the 128-byte swizzle
     float qscale;
     uint32_t a_bytes, kstage_bytes;  // a^K (or a^V) tile; one K-ring stage (b^K, a^K, a^V)
@@ -150,11 +157,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         const int depth = kside ? a.ks : kVS;
         uint64_t* full = kside ? k_full : v_full;
         uint64_t* empty = kside ? k_empty : v_empty;
+        // Shared basis: every b^V row (key j, rank s) is the value basis s, so the one
+        // V stage is loaded once (rows of keys 0..KT-1 of the table) and kept.
+        const int n_fill = (!kside && a.bcap == 0) ? min(n, 1) : n;
         if (lane == 0 && n > 0) {
             TileWalk<KT> tw;
             tw.init(P, g0);
             int i = 0;
-            for (; i < n && !*abort; ++i) {
+            for (; i < n_fill && !*abort; ++i) {
                 const int g = g0 + i;
                 tw.advance(P, g);
                 const int b = tw.b;
@@ -163,7 +173,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 if (i >= depth &&
                     !mbar_wait(&empty[s], (uint32_t)((i / depth - 1) & 1), lim, a.err, abort))
                     break;
-                const int y = (int)(((long long)b * a.cap + j0) * R);
+                const int y = (int)(((long long)b * a.bcap + j0) * R);
                 if (kside) {
                     // a^K, a^V: one TMA box each, 128-byte rows (one key at h 32, two at
                     // h 16) with the 128-byte swizzle; keys past the tensor read as zeros,
@@ -185,9 +195,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 } else {
                     // the value MMA has M = 128 rows of d_h: for d_h = 64 the one box is
                     // loaded twice and output rows 64..127 (a copy of 0..63) are dropped
+                    // (the kept shared-basis stage takes table rows 0..127: any KT keys'
+                    // rows are the same basis, and these exist whenever a key does)
+                    const int yv = a.bcap == 0 ? 0 : y;
                     mbar_arrive_expect_tx(&full[s], 2u * kBox);
-                    tma_load_2d(st_bv(s), &tmv, &full[s], 0, y);
-                    tma_load_2d(st_bv(s) + kBox, &tmv, &full[s], NB == 2 ? 64 : 0, y);
+                    tma_load_2d(st_bv(s), &tmv, &full[s], 0, yv);
+                    tma_load_2d(st_bv(s) + kBox, &tmv, &full[s], NB == 2 ? 64 : 0, yv);
                 }
             }
             for (int s = 0; s < depth; ++s) {                   // drain issued copies
@@ -218,8 +231,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 if (first && segp > 0 &&
                     !mbar_wait(o_free, (uint32_t)((segp - 1) & 1), lim, a.err, abort))
                     return false;
-                const int s = j % kVS;
-                if (!mbar_wait(&v_full[s], (uint32_t)((j / kVS) & 1), lim, a.err, abort)) return false;
+                const bool vkeep = a.bcap == 0;         // shared basis: one V stage, kept
+                const int s = vkeep ? 0 : j % kVS;
+                if (!mbar_wait(&v_full[s], vkeep ? 0u : (uint32_t)((j / kVS) & 1), lim, a.err, abort))
+                    return false;
                 tc_fence_after();
                 const uint32_t bv = smem_u32(st_bv(s));
                 const uint32_t wb = w0 + (uint32_t)(j & 1) * kQW;
@@ -231,7 +246,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                            idesc_pv, (first && k == 0) ? 0u : 1u);
                 }
                 mma_commit(&w_empty[j & 1]);
-                mma_commit(&v_empty[s]);
+                if (!vkeep) mma_commit(&v_empty[s]);
                 if (last) mma_commit(o_done);
                 return true;
             };
@@ -434,9 +449,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                         pack_bf16(w, wn);
                 }
             }
-            if (hg == 0 && !valid && j0 + jl >= len) {
+            if (hg == 0 && !valid && j0 + jl >= len && a.bcap != 0) {
                 // keys past the sequence: clear their b^V row (once the tile has landed)
-                // so 0 * (cache contents) = 0
+                // so 0 * (cache contents) = 0.  (The kept shared-basis stage holds finite
+                // basis rows and zero fill only, and is read by every tile.)
                 const int sv = i % kVS;
                 if (!bad) bad = !mbar_wait(&v_full[sv], (uint32_t)((i / kVS) & 1), lim, a.err, abort);
                 if (!bad) {
@@ -505,7 +521,8 @@ cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const D
     const size_t smem = fixed + (size_t)a.ks * a.kstage_bytes;
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
     CUtensorMap tmk, tmv;
-    const uint64_t dims[2] = {(uint64_t)DH, (uint64_t)c.batch * c.capacity * R};
+    // B rows: every sequence's (contextual), or one per-position table (shared basis)
+    const uint64_t dims[2] = {(uint64_t)DH, (uint64_t)(a.bcap ? c.batch : 1) * c.capacity * R};
     const uint64_t stride[1] = {(uint64_t)DH * 2};
     const uint32_t box[2] = {64, 128};
     if (!make_tmap_bf16(&tmk, c.b_k, 2, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 2, dims, stride, box))
@@ -555,6 +572,7 @@ cudaError_t launch_decode_tc(const Shape& s, const void* q_a, const void* q_b, c
     a.ws_o = ws + (size_t)plan.total_parts * s.H * 2;
     a.Rq = s.Rq;
     a.cap = c.capacity;
+    a.bcap = (int)b_seq_rows(s, c);
     a.qscale = 1.4426950408889634f / ((s.Rq > 0 ? (float)s.Rq : 1.f) * (float)s.Rk * std::sqrt((float)s.Dh));
     a.err = err;
     a.wait_limit = wait_limit;

@@ -20,6 +20,7 @@ struct PrefillArgs {
     const void *ca_k, *ca_v, *cb_k, *cb_v;
     void* out;
     int T, S, H, Dh, Rq, Rk, Rv, cap;
+    long long bcap;       // B_K / B_V rows between sequences: cap, or 0 (shared basis)
 };
 
 template <typename T>
@@ -44,26 +45,27 @@ __global__ void __launch_bounds__(128) prefill_simt_kernel(PrefillArgs a, SeqPar
     for (int u = 0; u < MAXU; ++u) {
         int e = lane + 32 * u;
         float v = 0.f;
-        if (e < a.Dh)
+        if (e < a.Dh) {
             if (a.Rq == 0)
                 v = to_f(bq[((long long)t * a.H + h) * a.Dh + e]);
             for (int r = 0; r < a.Rq; ++r)
                 v = fmaf(to_f(aq[((long long)t * a.H + h) * a.Rq + r]),
                          to_f(bq[((long long)t * a.Rq + r) * a.Dh + e]), v);
+        }
         q[u] = v * qscale;
         acc[u] = 0.f;
     }
     float m = -INFINITY, l = 0.f;
-    const long long seq_row = (long long)b * a.cap;
+    const long long seq_row = (long long)b * a.cap, bseq_row = (long long)b * a.bcap;
     for (int j = 0; j <= pos; ++j) {
-        const long long row = seq_row + j;
+        const long long row = seq_row + j, brow = bseq_row + j;
         float s = 0.f;
         for (int sk = 0; sk < a.Rk; ++sk) {
             float dot = 0.f;
 #pragma unroll
             for (int u = 0; u < MAXU; ++u) {
                 int e = lane + 32 * u;
-                if (e < a.Dh) dot = fmaf(q[u], to_f(bk[(row * a.Rk + sk) * a.Dh + e]), dot);
+                if (e < a.Dh) dot = fmaf(q[u], to_f(bk[(brow * a.Rk + sk) * a.Dh + e]), dot);
             }
             dot = warp_sum(dot);
             s = fmaf(to_f(ak[(row * a.H + h) * a.Rk + sk]), dot, s);
@@ -80,7 +82,7 @@ __global__ void __launch_bounds__(128) prefill_simt_kernel(PrefillArgs a, SeqPar
             if (e < a.Dh)
                 for (int sv = 0; sv < a.Rv; ++sv)
                     v = fmaf(to_f(av[(row * a.H + h) * a.Rv + sv]),
-                             to_f(bv[(row * a.Rv + sv) * a.Dh + e]), v);
+                             to_f(bv[(brow * a.Rv + sv) * a.Dh + e]), v);
             acc[u] = fmaf(acc[u], alpha, p * v);
         }
     }
@@ -102,7 +104,7 @@ cudaError_t launch_prefill_simt(const Shape& s, const tpa_factors& q, const tpa_
     a.ca_k = c.a_k; a.ca_v = c.a_v; a.cb_k = c.b_k; a.cb_v = c.b_v;
     a.out = out;
     a.T = batch * seqlen; a.S = seqlen; a.H = s.H; a.Dh = s.Dh;
-    a.Rq = s.Rq; a.Rk = s.Rk; a.Rv = s.Rv; a.cap = c.capacity;
+    a.Rq = s.Rq; a.Rk = s.Rk; a.Rv = s.Rv; a.cap = c.capacity; a.bcap = b_seq_rows(s, c);
     long long warps = (long long)a.T * a.H;
     long long blocks = (warps * 32 + 127) / 128;
     if (s.bf16)

@@ -30,6 +30,9 @@
 // setmaxnreg once the prologue is done.
 // TMEM: U double-buffered per M-block, U_{b,x} at 64*(2b+x); O_b at 256 + b*d_h.  W
 // overwrites the first half of U_{b,x} once the scores are read (bf16 pairs).
+// Shared basis (B_K, B_V shared across tokens, same page, 优点与创新 5): the b^K, b^V
+// tiles come from the layer's per-position tables, the same rows for every sequence
+// (read through L2), and only a^K, a^V are per sequence; nothing else changes.
 #include <algorithm>
 #include <cmath>
 
@@ -59,6 +62,7 @@ struct PrefillTcArgs {
     const __nv_bfloat16* ca_v;
     __nv_bfloat16* out;           // [T][H][DH]
     int S, H, Rq, cap, n_qblocks, qpb, stages;
+    int bcap;                     // B_K / B_V rows between sequences: cap, or 0 (shared basis)
     uint32_t a_bytes;             // bytes of one a^K (or a^V) tile: KT*H*R*2
     uint32_t stage_bytes;
     float qscale, out_scale;
@@ -418,13 +422,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 const int rows_a = min(KT, a.cap - j0);
                 const uint32_t abytes = (uint32_t)rows_a * H * R * 2u;
                 mbar_arrive_expect_tx(&kv_full[s], full_bytes + 2u * abytes);
-                const int y = (int)(((long long)b * a.cap + j0) * R);
+                const int yb = b * a.bcap + j0;             // B row of key j0
+                const int y = yb * R;
 #pragma unroll
                 for (int cb = 0; cb < NB; ++cb) {
                     if constexpr (PK) {
                         // rank-major box: (column, key, rank) = (cb*64, key of j0, 0)
-                        tma_load_3d(stage_bk(s) + cb * kBox, &tmk, &kv_full[s], cb * 64, b * a.cap + j0, 0);
-                        tma_load_3d(stage_bv(s) + cb * kBox, &tmv, &kv_full[s], cb * 64, b * a.cap + j0, 0);
+                        tma_load_3d(stage_bk(s) + cb * kBox, &tmk, &kv_full[s], cb * 64, yb, 0);
+                        tma_load_3d(stage_bv(s) + cb * kBox, &tmv, &kv_full[s], cb * 64, yb, 0);
                     } else {
                         tma_load_2d(stage_bk(s) + cb * kBox, &tmk, &kv_full[s], cb * 64, y);
                         tma_load_2d(stage_bv(s) + cb * kBox, &tmv, &kv_full[s], cb * 64, y);
@@ -746,16 +751,18 @@ cudaError_t launch_t(const PrefillTcArgs& a0, const tpa_cache& c, int batch, con
     a.stages = std::min(8, (int)(budget / a.stage_bytes));
     if (a.stages < 3) return cudaErrorInvalidValue;   // QK(t+2) and PV(t) use different stages
     CUtensorMap tmk, tmv;
+    // B rows: every sequence's (contextual), or one per-position table (shared basis)
+    const uint64_t b_keys = (uint64_t)(a.bcap ? c.batch : 1) * (uint64_t)c.capacity;
     if constexpr (R == 2 && HC == 16) {
         // packed path: [d_h][key][rank] with rank outermost, so a box of KT keys x 2
         // ranks lands rank-major (row s*KT + key)
-        const uint64_t dims[3] = {(uint64_t)DH, (uint64_t)c.batch * c.capacity, (uint64_t)R};
+        const uint64_t dims[3] = {(uint64_t)DH, b_keys, (uint64_t)R};
         const uint64_t stride[2] = {(uint64_t)R * DH * 2, (uint64_t)DH * 2};
         const uint32_t box[3] = {64, (uint32_t)KT, (uint32_t)R};
         if (!make_tmap_bf16(&tmk, c.b_k, 3, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 3, dims, stride, box))
             return cudaErrorInvalidValue;
     } else {
-        const uint64_t dims[2] = {(uint64_t)DH, (uint64_t)c.batch * c.capacity * R};
+        const uint64_t dims[2] = {(uint64_t)DH, b_keys * R};
         const uint64_t stride[1] = {(uint64_t)DH * 2};
         const uint32_t box[2] = {64, (uint32_t)kUW};
         if (!make_tmap_bf16(&tmk, c.b_k, 2, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 2, dims, stride, box))
@@ -799,6 +806,7 @@ cudaError_t launch_prefill_tc(const Shape& s, const tpa_factors& q, const tpa_ca
     a.H = s.H;
     a.Rq = s.Rq;
     a.cap = c.capacity;
+    a.bcap = (int)b_seq_rows(s, c);
     a.qpb = 256 / s.H;
     a.n_qblocks = (seqlen + a.qpb - 1) / a.qpb;
     a.qscale = 1.4426950408889634f / ((float)(s.Rq > 0 ? s.Rq : 1) * (float)s.Rk * std::sqrt((float)s.Dh));

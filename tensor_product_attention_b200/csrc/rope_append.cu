@@ -7,7 +7,13 @@
 //
 // Cache append: cache[:bsz, start_pos:start_pos+seqlen] = factors from the same forward,
 // done as one bit-exact, 16-byte vectorised, coalesced copy of the four cached factor
-// tensors; HBM-bound (reads and writes (R_K+R_V)(h+d_h) elements per token).
+// tensors; HBM-bound (reads and writes (R_K+R_V)(h+d_h) elements per token).  With a
+// shared basis only A_K and A_V are per token, so only those two are copied.
+//
+// Shared-basis tables: the variant that shares the basis vectors across tokens (same
+// page, 优点与创新 5) keeps B_K and B_V as layer parameters.  Its cache side is one
+// table per layer, row p = the key basis rotated at position p (pre-rotated as B_K is
+// cached, 关键问题及回答 问题2) and the value basis, which every sequence reads.
 #include "tpa_internal.h"
 #include "device_util.cuh"
 
@@ -71,11 +77,12 @@ cudaError_t launch_cache_append(const Shape& s, const tpa_cache& c, const tpa_fa
                                 int batch, int n_tokens, const SeqParams& start,
                                 cudaStream_t st) {
     const int es = s.bf16 ? 2 : 4;
+    const int n_arr = s.shared ? 2 : 4;       // shared basis: A_K, A_V only
     long long row_bytes[4] = {(long long)s.H * s.Rk * es, (long long)s.H * s.Rv * es,
                               (long long)s.Rk * s.Dh * es, (long long)s.Rv * s.Dh * es};
     // widest vector that divides every row (pointers are 16-byte aligned by contract)
     int vec = 16;
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < n_arr; ++i)
         while (row_bytes[i] % vec) vec >>= 1;
     AppendArgs a;
     a.src[0] = (const char*)kv.a_k; a.src[1] = (const char*)kv.a_v;
@@ -85,7 +92,7 @@ cudaError_t launch_cache_append(const Shape& s, const tpa_cache& c, const tpa_fa
     for (int i = 0; i < 4; ++i) a.row_units[i] = row_bytes[i] / vec;
     a.batch = batch; a.n_tokens = n_tokens; a.capacity = c.capacity; a.lengths = c.lengths;
     long long most = 0;
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < n_arr; ++i) {
         long long t = (long long)batch * n_tokens * a.row_units[i];
         if (t > most) most = t;
     }
@@ -93,13 +100,59 @@ cudaError_t launch_cache_append(const Shape& s, const tpa_cache& c, const tpa_fa
     long long blocks = (most + threads - 1) / threads;
     if (blocks > 148 * 16) blocks = 148 * 16;
     if (blocks < 1) blocks = 1;
-    dim3 grid((unsigned)blocks, 4);
+    dim3 grid((unsigned)blocks, (unsigned)n_arr);
     switch (vec) {
         case 16: append_kernel<uint4><<<grid, threads, 0, st>>>(a, start); break;
         case 8: append_kernel<uint2><<<grid, threads, 0, st>>>(a, start); break;
         case 4: append_kernel<uint32_t><<<grid, threads, 0, st>>>(a, start); break;
         default: append_kernel<uint16_t><<<grid, threads, 0, st>>>(a, start); break;
     }
+    return cudaGetLastError();
+}
+
+// table_k[p][s][2k, 2k+1] = basis_k[s] pair k turned by cs[p][k] (the rotation and the
+// fp32 arithmetic of the projection epilogue's RoPE); table_v[p][s][:] = basis_v[s].
+template <typename T>
+__global__ void basis_table_kernel(const T* __restrict__ bk, const T* __restrict__ bv,
+                                   const float2* __restrict__ cs, int capacity, int Rk, int Rv,
+                                   int half, T* __restrict__ tk, T* __restrict__ tv) {
+    const long long step = (long long)gridDim.x * blockDim.x;
+    const long long t0 = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    const int d = 2 * half;
+    const long long nk = (long long)capacity * Rk * half;
+    for (long long u = t0; u < nk; u += step) {
+        const int k = (int)(u % half);
+        const long long ps = u / half;             // p * Rk + s
+        const int sr = (int)(ps % Rk);
+        const int p = (int)(ps / Rk);
+        const float x0 = to_f(bk[(long long)sr * d + 2 * k]);
+        const float x1 = to_f(bk[(long long)sr * d + 2 * k + 1]);
+        const float2 r = cs[(long long)p * half + k];
+        tk[ps * d + 2 * k] = from_f<T>(x0 * r.x - x1 * r.y);
+        tk[ps * d + 2 * k + 1] = from_f<T>(x0 * r.y + x1 * r.x);
+    }
+    const long long nv = (long long)capacity * Rv * d;
+    const long long per = (long long)Rv * d;
+    for (long long u = t0; u < nv; u += step) tv[u] = bv[u % per];
+}
+
+cudaError_t launch_shared_basis_tables(const Shape& s, const void* basis_k, const void* basis_v,
+                                       const float* cs, int capacity, void* table_k,
+                                       void* table_v, cudaStream_t st) {
+    const long long work = (long long)capacity * (s.Rk * s.Dh / 2 + s.Rv * s.Dh);
+    long long blocks = (work + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    const float2* c2 = reinterpret_cast<const float2*>(cs);
+    if (s.bf16)
+        basis_table_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(basis_k), static_cast<const __nv_bfloat16*>(basis_v), c2,
+            capacity, s.Rk, s.Rv, s.Dh / 2, static_cast<__nv_bfloat16*>(table_k),
+            static_cast<__nv_bfloat16*>(table_v));
+    else
+        basis_table_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(
+            static_cast<const float*>(basis_k), static_cast<const float*>(basis_v), c2, capacity,
+            s.Rk, s.Rv, s.Dh / 2, static_cast<float*>(table_k), static_cast<float*>(table_v));
     return cudaGetLastError();
 }
 

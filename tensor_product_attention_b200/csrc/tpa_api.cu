@@ -48,6 +48,7 @@ tpa_status check_dims(const tpa_dims* d, bool need_q) {
     if (d->dtype != TPA_F32 && d->dtype != TPA_BF16) return TPA_ERR_INVALID;
     if (d->n_heads < 1 || d->head_dim < 2 || (d->head_dim & 1)) return TPA_ERR_INVALID;
     if (d->rank_k < 1 || d->rank_v < 1 || d->rank_q < 0) return TPA_ERR_INVALID;
+    if (d->shared_basis != 0 && d->shared_basis != 1) return TPA_ERR_INVALID;
     if (need_q && d->rank_q < 1) return TPA_ERR_UNSUPPORTED;
     if (d->n_heads > 4096 || d->head_dim > 4096 || d->rank_q > 256 || d->rank_k > 256 ||
         d->rank_v > 256)
@@ -130,7 +131,8 @@ const char* tpa_status_string(tpa_status s) {
 size_t tpa_cache_bytes_per_token(const tpa_dims* d) {
     if (check_dims(d, false) != TPA_OK) return 0;
     size_t es = d->dtype == TPA_BF16 ? 2 : 4;
-    return (size_t)(d->rank_k + d->rank_v) * (size_t)(d->n_heads + d->head_dim) * es;
+    const size_t per_rank = (size_t)d->n_heads + (d->shared_basis ? 0 : (size_t)d->head_dim);
+    return (size_t)(d->rank_k + d->rank_v) * per_rank * es;
 }
 
 void tpa_set_wait_limit(uint32_t polls) { g_wait_limit.store(polls); }
@@ -151,8 +153,9 @@ tpa_status tpa_project(const tpa_dims* d, const void* x, const void* w_cat, int3
     if (st != TPA_OK) return st;
     if (d->d_model < 1) return TPA_ERR_INVALID;
     if (!x || !w_cat || !start_pos || !rope_cs || !out) return TPA_ERR_INVALID;
-    if ((d->rank_q > 0 && !out->a_q) || !out->b_q || !out->a_k || !out->b_k || !out->a_v || !out->b_v)
+    if ((d->rank_q > 0 && !out->a_q) || !out->b_q || !out->a_k || !out->a_v)
         return TPA_ERR_INVALID;
+    if (!d->shared_basis && (!out->b_k || !out->b_v)) return TPA_ERR_INVALID;
     if (!aligned16(x) || !aligned16(w_cat) || !aligned16(rope_cs)) return TPA_ERR_INVALID;
     if (batch < 1 || batch > TPA_MAX_BATCH || seqlen < 1 || max_pos < 1)
         return TPA_ERR_INVALID;
@@ -176,10 +179,10 @@ tpa_status tpa_cache_append(const tpa_dims* d, const tpa_cache* c, const tpa_fac
     tpa_status st = check_dims(d, false);
     if (st != TPA_OK) return st;
     if ((st = check_cache(c, batch)) != TPA_OK) return st;
-    if (!kv || !kv->a_k || !kv->a_v || !kv->b_k || !kv->b_v || !start_pos)
-        return TPA_ERR_INVALID;
-    if (!aligned16(kv->a_k) || !aligned16(kv->a_v) || !aligned16(kv->b_k) ||
-        !aligned16(kv->b_v))
+    if (!kv || !kv->a_k || !kv->a_v || !start_pos) return TPA_ERR_INVALID;
+    if (!aligned16(kv->a_k) || !aligned16(kv->a_v)) return TPA_ERR_INVALID;
+    if (!d->shared_basis &&
+        (!kv->b_k || !kv->b_v || !aligned16(kv->b_k) || !aligned16(kv->b_v)))
         return TPA_ERR_INVALID;
     if (n_tokens < 1) return TPA_ERR_INVALID;
     SeqParams sp;
@@ -190,6 +193,24 @@ tpa_status tpa_cache_append(const tpa_dims* d, const tpa_cache* c, const tpa_fac
     }
     return launched(launch_cache_append(shape_of(*d), *c, *kv, batch, n_tokens, sp,
                                         (cudaStream_t)stream));
+}
+
+tpa_status tpa_shared_basis_tables(const tpa_dims* d, const void* basis_k, const void* basis_v,
+                                   const float* rope_cs, int32_t max_pos, int32_t capacity,
+                                   void* table_k, void* table_v, tpa_stream_t stream) {
+    tpa_status st = check_dims(d, false);
+    if (st != TPA_OK) return st;
+    if (!d->shared_basis) return TPA_ERR_INVALID;
+    if (!basis_k || !basis_v || !rope_cs || !table_k || !table_v) return TPA_ERR_INVALID;
+    if (!aligned16(basis_k) || !aligned16(basis_v) || !aligned16(rope_cs) ||
+        !aligned16(table_k) || !aligned16(table_v))
+        return TPA_ERR_INVALID;
+    if (capacity < 1 || max_pos < 1) return TPA_ERR_INVALID;
+    if (capacity > max_pos) return TPA_ERR_CAPACITY;
+    if ((long long)capacity * (d->rank_k + d->rank_v) * d->head_dim > (1LL << 40))
+        return TPA_ERR_UNSUPPORTED;
+    return launched(launch_shared_basis_tables(shape_of(*d), basis_k, basis_v, rope_cs, capacity,
+                                               table_k, table_v, (cudaStream_t)stream));
 }
 
 tpa_status tpa_prefill(const tpa_dims* d, const tpa_factors* q, const tpa_cache* c,

@@ -18,16 +18,24 @@ struct SeqParams {
 struct Shape {
     int D, H, Dh, Rq, Rk, Rv;
     bool bf16;
+    bool shared;    // shared basis: B_K, B_V are per-position tables, one for all sequences
 };
 
 inline Shape shape_of(const tpa_dims& d) {
     return Shape{d.d_model, d.n_heads, d.head_dim, d.rank_q, d.rank_k, d.rank_v,
-                 d.dtype == TPA_BF16};
+                 d.dtype == TPA_BF16, d.shared_basis != 0};
+}
+
+// Cache rows between sequences in the B_K / B_V tensors: the capacity, or 0 for a
+// shared basis (every sequence reads the same per-position table).
+inline long long b_seq_rows(const Shape& s, const tpa_cache& c) {
+    return s.shared ? 0 : (long long)c.capacity;
 }
 
 // Column layout of the stacked projection output: [a_q | a_k | a_v | b_q | b_k | b_v].
 // TPA-KVonly (rank_q = 0): a_q is empty and the b_q segment is the plain query
-// projection, h rows of d_h ([T][h][d_h]), rotated like B_Q.
+// projection, h rows of d_h ([T][h][d_h]), rotated like B_Q.  Shared basis: the b_k
+// and b_v segments are empty (no column maps to them).
 struct ProjLayout {
     int off[7];    // segment starts, off[6] = N
     void* dst[6];  // a_q, a_k, a_v, b_q, b_k, b_v
@@ -46,7 +54,8 @@ __host__ __device__ inline long long seg_row(const ProjLayout& L, int s, long lo
 inline ProjLayout proj_layout(const Shape& s, const tpa_factors& f) {
     ProjLayout L;
     const int q_rows = s.Rq > 0 ? s.Rq : s.H;
-    int w[6] = {s.H * s.Rq, s.H * s.Rk, s.H * s.Rv, q_rows * s.Dh, s.Rk * s.Dh, s.Rv * s.Dh};
+    int w[6] = {s.H * s.Rq, s.H * s.Rk, s.H * s.Rv, q_rows * s.Dh,
+                s.shared ? 0 : s.Rk * s.Dh, s.shared ? 0 : s.Rv * s.Dh};
     L.off[0] = 0;
     for (int i = 0; i < 6; ++i) L.off[i + 1] = L.off[i] + w[i];
     L.dst[0] = f.a_q; L.dst[1] = f.a_k; L.dst[2] = f.a_v;
@@ -89,6 +98,10 @@ cudaError_t launch_project_tc(const Shape& s, const void* x, const void* w, int 
                               const ProjLayout& L, int* err, uint32_t wait_limit,
                               cudaStream_t st);
 bool project_tc_supported(const Shape& s, int T);
+
+cudaError_t launch_shared_basis_tables(const Shape& s, const void* basis_k, const void* basis_v,
+                                       const float* cs, int capacity, void* table_k,
+                                       void* table_v, cudaStream_t st);
 
 cudaError_t launch_cache_append(const Shape& s, const tpa_cache& c, const tpa_factors& kv,
                                 int batch, int n_tokens, const SeqParams& start,

@@ -25,7 +25,7 @@ def rel_err(gpu, ref) -> float:
 
 def dims_of(wl, binding):
     return binding.Dims(wl.d_model, wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v,
-                        binding.BF16 if wl.dtype == "bf16" else binding.F32)
+                        binding.BF16 if wl.dtype == "bf16" else binding.F32, int(wl.shared_basis))
 
 
 def fill_cache(cache, b, seq: dict, start: int = 0):

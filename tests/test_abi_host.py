@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(bnd):
 
 
 def test_abi_version_and_status_strings(bnd):
-    assert bnd.tpa_abi_version() == 1
+    assert bnd.tpa_abi_version() == 2
     assert "sm_100a" in bnd.tpa_build_info()
     for code in range(7):
         assert bnd._lib.tpa_status_string(code)
@@ -138,3 +138,28 @@ def test_workspace_size_formula(bnd):
     per_part = 16 * (128 + 2) * 4
     assert n % per_part == 0
     assert 64 * per_part <= n <= (64 + 1024) * per_part
+
+
+def test_shared_basis_host_validation(bnd):
+    # shared basis: only A_K, A_V per token, (R_K + R_V) h elements
+    sh = bnd.Dims(64, 16, 128, 6, 2, 2, bnd.BF16, 1)
+    assert bnd.tpa_cache_bytes_per_token(sh) == (2 + 2) * 16 * 2
+    assert bnd.tpa_cache_bytes_per_token(bnd.Dims(64, 16, 128, 6, 2, 2, bnd.BF16, 2)) == 0
+    assert sh.n_proj == 16 * (6 + 2 + 2) + 6 * 128
+    by = ctypes.byref
+    fake = 0x10000                      # aligned, never dereferenced: validation fails first
+    d = sh.c()
+    tables = bnd._lib.tpa_shared_basis_tables
+    ctx = bnd.Dims(64, 16, 128, 6, 2, 2, bnd.BF16, 0).c()
+    assert tables(by(ctx), fake, fake, fake, 64, 64, fake, fake, None) == 1      # not shared
+    assert tables(by(d), None, fake, fake, 64, 64, fake, fake, None) == 1
+    assert tables(by(d), fake, fake, fake, 64, 64, fake + 8, fake, None) == 1   # misaligned
+    assert tables(by(d), fake, fake, fake, 64, 0, fake, fake, None) == 1        # no capacity
+    assert tables(by(d), fake, fake, fake, 64, 65, fake, fake, None) == 3       # past RoPE table
+    # projection: shared layers need no B_K / B_V outputs, but still the A factors
+    f = bnd.tpa_factors(fake, fake, None, None, None, None)
+    assert bnd._lib.tpa_project(by(d), fake, fake, 1, 1, bnd._ints([0]), fake, 8, by(f), None) == 1
+    # append: A factors are still required
+    cache = bnd.tpa_cache(fake, fake, fake, fake, fake, 1, 8)
+    assert bnd._lib.tpa_cache_append(by(d), by(cache), by(f), 1, 1, bnd._ints([0]), None) == 1
+    assert bnd._lib.tpa_cache_append(by(d), by(cache), by(f), 1, 1, bnd._ints([8]), None) == 1

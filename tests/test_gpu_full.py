@@ -62,6 +62,14 @@ def _full_decode(tpa, wl, sample):
     lengths = [int(v) for v in I.decode_lengths(wl)]
     B = wl.batch
     cache = tpa.alloc_cache(dims, B, max(lengths))
+    basis = None
+    if wl.shared_basis:
+        basis = I.shared_basis(wl)
+        cs = torch.empty((max(lengths), wl.head_dim // 2, 2), dtype=torch.float32, device="cuda")
+        tpa.tpa_rope_table(dims, wl.rope_base, max(lengths), cs)
+        tpa.tpa_shared_basis_tables(dims, basis["b_k"].cuda(), basis["b_v"].cuda(), cs, max(lengths),
+                                    cache.b_k, cache.b_v)
+        del cs
     q_parts = {}
     for b, L in enumerate(lengths):
         seq = I.decode_sequence(wl, b, L)
@@ -80,9 +88,13 @@ def _full_decode(tpa, wl, sample):
     torch.cuda.synchronize()
     assert tpa.tpa_get_device_error() == 0
     od = oracle_dims(wl)
+    tab = None
+    if basis is not None:
+        tab = oracle.shared_basis_tables({n: f64(t) for n, t in basis.items()}, od, max(lengths), wl.rope_base)
     for b in sample:
         seq = {k: f64(v) for k, v in I.decode_sequence(wl, b, lengths[b]).items()}
-        err = rel_err(out[b], oracle.decode_attention(seq, seq, od, lengths[b]))
+        kv = seq if tab is None else {"a_k": seq["a_k"], "a_v": seq["a_v"], **tab}
+        err = rel_err(out[b], oracle.decode_attention(seq, kv, od, lengths[b]))
         assert err < TOL["bf16"], (b, lengths[b], err)
 
 
@@ -95,3 +107,8 @@ def test_full_kvonly_decode_b16_ctx64k_128k(tpa):
     wl = I.WORKLOADS["kvonly_decode_b16_ctx64k_128k"]
     lengths = I.decode_lengths(wl)
     _full_decode(tpa, wl, [int(np.argmin(lengths)), int(np.argmax(lengths))])
+
+
+def test_full_shared_basis_decode_b64_ctx32k(tpa):
+    wl = I.WORKLOADS["shared_basis_decode_b64_ctx32k"]
+    _full_decode(tpa, wl, [0, 41, wl.batch - 1])
