@@ -40,6 +40,7 @@ METRIC = "TPA decode factor-cache GB/s (% HBM peak); prefill TFLOP/s (% bf16 pea
 DEFAULT = "prefill_b8_s2048_d1024"
 DECODE_LEG = "decode_b64_ctx32k"
 KVONLY_DECODE_LEG = "kvonly_decode_b16_ctx64k_128k"
+SHARED_DECODE_LEG = "shared_basis_decode_b64_ctx32k"
 FLUSH_BYTES = 256 << 20          # > 126 MB L2
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture of
@@ -70,6 +71,8 @@ def proj_flops(wl, tokens: int) -> int:
     n = (wl.rank_q + wl.rank_k + wl.rank_v) * (wl.n_heads + wl.head_dim)
     if wl.rank_q == 0:
         n += wl.n_heads * wl.head_dim              # TPA-KVonly: the plain W_Q
+    if wl.shared_basis:
+        n -= (wl.rank_k + wl.rank_v) * wl.head_dim  # no W_B_k, W_B_v
     return 2 * tokens * n * wl.d_model
 
 
@@ -78,8 +81,11 @@ def causal_pairs(batch: int, S: int, start: int = 0) -> int:
 
 
 def cache_bytes_per_token(wl) -> int:
+    """Per-token cache bytes: (R_K + R_V)(h + d_h) elements, or (R_K + R_V) h with a
+    shared basis (its B side is one per-layer table, counted once per launch)."""
     es = 2 if wl.dtype == "bf16" else 4
-    return (wl.rank_k + wl.rank_v) * (wl.n_heads + wl.head_dim) * es
+    per_rank = wl.n_heads + (0 if wl.shared_basis else wl.head_dim)
+    return (wl.rank_k + wl.rank_v) * per_rank * es
 
 
 def peaks():
@@ -287,14 +293,25 @@ class DecodeStep:
     def __init__(self, wl, tpa):
         self.wl, self.tpa = wl, tpa
         self.dims = tpa.Dims(0, wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v,
-                             tpa.BF16 if wl.dtype == "bf16" else tpa.F32)
+                             tpa.BF16 if wl.dtype == "bf16" else tpa.F32, int(wl.shared_basis))
         self.lengths = [int(v) for v in I.decode_lengths(wl)]
         B = wl.batch
         self.cache = tpa.alloc_cache(self.dims, B, max(self.lengths))
+        if wl.shared_basis:
+            # the layer's per-position basis tables: built once, like the weights
+            cap = max(self.lengths)
+            basis = I.shared_basis(wl)
+            cs = torch.empty((cap, wl.head_dim // 2, 2), dtype=torch.float32, device="cuda")
+            tpa.tpa_rope_table(self.dims, wl.rope_base, cap, cs)
+            tpa.tpa_shared_basis_tables(self.dims, basis["b_k"].cuda(), basis["b_v"].cuda(), cs, cap,
+                                        self.cache.b_k, self.cache.b_v)
+            torch.cuda.synchronize()
+            del cs
+        per_seq = ("a_k", "a_v") if wl.shared_basis else ("a_k", "a_v", "b_k", "b_v")
         qa, qb = [], []
         for b, L in enumerate(self.lengths):
             seq = I.decode_sequence(wl, b, L)
-            for n in ("a_k", "a_v", "b_k", "b_v"):
+            for n in per_seq:
                 getattr(self.cache, n)[b, :L].copy_(seq[n])
             if wl.rank_q:
                 qa.append(seq["a_q"]); qb.append(seq["b_q"])
@@ -312,7 +329,14 @@ class DecodeStep:
         self.launches_per_step = 2   # decode, combine
 
     def factor_bytes(self):
-        return sum(self.lengths) * cache_bytes_per_token(self.wl)
+        """Cache bytes one launch must read: every key's factors, plus (shared basis)
+        the key table rows up to the longest context and one value tile, once."""
+        n = sum(self.lengths) * cache_bytes_per_token(self.wl)
+        if self.wl.shared_basis:
+            es = 2 if self.wl.dtype == "bf16" else 4
+            n += max(self.lengths) * self.wl.rank_k * self.wl.head_dim * es
+            n += self.wl.rank_v * self.wl.head_dim * es
+        return n
 
     def bytes(self):
         q = self.q_b.numel() * self.q_b.element_size() + (0 if self.q_a is None else self.q_a.numel() * self.q_a.element_size())
@@ -421,11 +445,13 @@ def oracle_prefill_sample(wl, n_seq: int = 1, seqlen: int | None = None):
     sequences of the workload; returns (seconds, flops of that sample)."""
     import oracle
     S = seqlen or wl.seqlen
-    od = oracle.Dims(wl.d_model, wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v)
+    od = oracle.Dims(wl.d_model, wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v,
+                     shared_basis=wl.shared_basis)
+    basis = {k: v.double().numpy() for k, v in I.shared_basis(wl).items()} if wl.shared_basis else None
     x = np.stack([I.prefill_x(wl, b, S).double().numpy() for b in range(n_seq)])
     w = I.prefill_w(wl).double().numpy()
     t0 = time.perf_counter()
-    oracle.tpa_forward(x, w, od, wl.rope_base)
+    oracle.tpa_forward(x, w, od, wl.rope_base, basis=basis)
     dt = time.perf_counter() - t0
     return dt, proj_flops(wl, n_seq * S) + attn_flops_per_pair(wl) * causal_pairs(n_seq, S)
 
@@ -433,7 +459,8 @@ def oracle_prefill_sample(wl, n_seq: int = 1, seqlen: int | None = None):
 def oracle_decode_sample(wl, n_seq: int = 1, length: int | None = None):
     """Time the oracle's decode on n_seq sequences; returns (seconds, factor bytes)."""
     import oracle
-    od = oracle.Dims(0, wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v)
+    od = oracle.Dims(0, wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v,
+                     shared_basis=wl.shared_basis)
     lengths = I.decode_lengths(wl)
     total = 0
     seqs = []
@@ -441,9 +468,13 @@ def oracle_decode_sample(wl, n_seq: int = 1, length: int | None = None):
         L = int(length or lengths[b])
         seqs.append(({k: v.double().numpy() for k, v in I.decode_sequence(wl, b, L).items()}, L))
         total += L * cache_bytes_per_token(wl)
+    basis = {k: v.double().numpy() for k, v in I.shared_basis(wl).items()} if wl.shared_basis else None
     t0 = time.perf_counter()
     for s, L in seqs:
-        oracle.decode_attention(s, s, od, L)
+        kv = s
+        if basis is not None:       # the per-layer tables are part of the timed work
+            kv = {"a_k": s["a_k"], "a_v": s["a_v"], **oracle.shared_basis_tables(basis, od, L, wl.rope_base)}
+        oracle.decode_attention(s, kv, od, L)
     return time.perf_counter() - t0, total
 
 
@@ -579,7 +610,8 @@ def main():
 
     # the decode configurations ride along with the prefill step as separate legs
     legs_to_run = [] if (wl.kind != "prefill" or args.no_decode_leg) else \
-        [("decode_leg", DECODE_LEG), ("kvonly_decode_leg", KVONLY_DECODE_LEG)]
+        [("decode_leg", DECODE_LEG), ("kvonly_decode_leg", KVONLY_DECODE_LEG),
+         ("shared_basis_decode_leg", SHARED_DECODE_LEG)]
     for key, name in legs_to_run:
         dl = I.WORKLOADS[name]
         dstep = DecodeStep(dl, tpa)

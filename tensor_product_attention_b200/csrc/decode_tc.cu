@@ -20,15 +20,18 @@
 // only revisits it (rescaling O^T in tensor memory) when a score exceeds it by more
 // than 2^8, so a tile normally needs one pass and one barrier.
 //
-// Warp roles: warp 0 TMA (two stages of b^K/b^V tiles, 128-byte swizzle, and a^K/a^V
-// bulk copies), warp 1 TMEM owner and MMA issuer, warps 2.. softmax (4 warps per 16
-// heads; TMEM lane = row).  TMEM: U^T double-buffered (2 x h columns) and O^T (h).
+// Warp roles: warp 0 TMA for the K ring (b^K tiles, 128-byte swizzle, and a^K/a^V),
+// warp 2 TMA for the V ring (b^V tiles), warp 1 TMEM owner and QK issuer, warp 3 PV
+// issuer, warps 4.. softmax (4 warps per 16 heads; TMEM lane = row).  TMEM: U^T
+// double-buffered (2 x h columns) and O^T (h).
 //
-// Shared basis (B_K, B_V shared across tokens, same page, 优点与创新 5): b^K tiles come
-// from the layer's per-position table (row j = the key basis rotated at j, the same for
-// every sequence, so it is read through L2), and every b^V row of a tile is the value
-// basis, so one V stage is loaded once and reused by every PV.  Per key only the
-// (R_K + R_V) h A factors come from the sequence's cache.
+// Shared basis (B_K, B_V shared across tokens, same page, 优点与创新 5), kernel SB: b^K
+// tiles come from the layer's per-position table (row j = the key basis rotated at j,
+// the same for every sequence, so it is read through L2).  Every value row of rank s is
+// the basis b^V_s, so O_h = sum_s (sum_j p_{j,h} a^V_{j,h,s}) b^V_s: the softmax threads
+// keep sum_j p a^V in registers (each row has one rank) and apply the basis once per
+// part; there is no PV MMA, no V ring and no W^T.  Per key only the (R_K + R_V) h A
+// factors come from the sequence's cache.
 #include <algorithm>
 #include <cmath>
 
@@ -50,6 +53,7 @@ struct DecodeTcArgs {
     const __nv_bfloat16* q_b;      // [B][Rq][DH] or q [B][H][DH]
     const __nv_bfloat16* ca_k;     // [B][cap][H][R]
     const __nv_bfloat16* ca_v;
+    const __nv_bfloat16* cb_v;     // shared basis: the value table (row 0 = the basis)
     float* ws_ml;                  // [parts][H][2]
     float* ws_o;                   // [parts][H][DH]
     int Rq, cap;
@@ -75,8 +79,8 @@ struct TileWalk {
     }
 };
 
-template <int DH, int HH, int R>
-__global__ void __launch_bounds__(96 + 32 * 4 * (HH / 16), 1)
+template <int DH, int HH, int R, bool SB>
+__global__ void __launch_bounds__(128 + 32 * 4 * (HH / 16), 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                  const __grid_constant__ CUtensorMap tmak, const __grid_constant__ CUtensorMap tmav,
                  const DecodeTcArgs a, const DecodePlan P) {
@@ -91,12 +95,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                                                ~uintptr_t(1023));
     // Two rings: K (b^K, a^K, a^V: read by QK and the softmax) a.ks deep, and V (b^V:
     // read by PV) kVS deep, so the key side prefetches further than the value side.
+    // The shared-basis kernel (SB) has no V ring and no W^T buffers.
     uint8_t* kring = smem;
     uint8_t* vring = kring + (size_t)a.ks * a.kstage_bytes;
-    uint8_t* qbuf = vring + (size_t)kVS * 2 * kBox;                 // 2 x q~
-    uint8_t* wbuf = qbuf + 2 * kQW;                                 // 2 x W^T
-    float* red = reinterpret_cast<float*>(wbuf + 2 * kQW);          // [NG][4][16] scratch
-    uint64_t* bars = reinterpret_cast<uint64_t*>(red + NG * 64);
+    uint8_t* qbuf = vring + (SB ? (size_t)0 : (size_t)kVS * 2 * kBox);   // 2 x q~
+    uint8_t* wbuf = qbuf + 2 * kQW;                                     // 2 x W^T
+    float* red = reinterpret_cast<float*>(wbuf + (SB ? 0u : 2 * kQW));  // [NG][192] scratch
+    uint64_t* bars = reinterpret_cast<uint64_t*>(red + NG * 192);
     uint64_t* k_full = bars;                     // [ks]
     uint64_t* k_empty = k_full + a.ks;           // [ks] every softmax thread is done with it
     uint64_t* v_full = k_empty + a.ks;           // [kVS]
@@ -136,7 +141,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         }
         mbar_init(o_done, 1);
         mbar_init(o_free, NSM);
-        mbar_init(fin, 1);
+        mbar_init(fin, SB ? 1 : 2);              // one commit from each MMA issuer
         *abort = 0;
         fence_mbar_init();
     }
@@ -150,21 +155,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0 || warp == 2) {
+    if (warp == 0 || (warp == 2 && !SB)) {
         // ---------------------------------------------------------------- producers
         // warp 0: the K ring (b^K, a^K, a^V); warp 2: the V ring (b^V)
         const bool kside = warp == 0;
         const int depth = kside ? a.ks : kVS;
         uint64_t* full = kside ? k_full : v_full;
         uint64_t* empty = kside ? k_empty : v_empty;
-        // Shared basis: every b^V row (key j, rank s) is the value basis s, so the one
-        // V stage is loaded once (rows of keys 0..KT-1 of the table) and kept.
-        const int n_fill = (!kside && a.bcap == 0) ? min(n, 1) : n;
         if (lane == 0 && n > 0) {
             TileWalk<KT> tw;
             tw.init(P, g0);
             int i = 0;
-            for (; i < n_fill && !*abort; ++i) {
+            for (; i < n && !*abort; ++i) {
                 const int g = g0 + i;
                 tw.advance(P, g);
                 const int b = tw.b;
@@ -195,12 +197,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 } else {
                     // the value MMA has M = 128 rows of d_h: for d_h = 64 the one box is
                     // loaded twice and output rows 64..127 (a copy of 0..63) are dropped
-                    // (the kept shared-basis stage takes table rows 0..127: any KT keys'
-                    // rows are the same basis, and these exist whenever a key does)
-                    const int yv = a.bcap == 0 ? 0 : y;
                     mbar_arrive_expect_tx(&full[s], 2u * kBox);
-                    tma_load_2d(st_bv(s), &tmv, &full[s], 0, yv);
-                    tma_load_2d(st_bv(s) + kBox, &tmv, &full[s], NB == 2 ? 64 : 0, yv);
+                    tma_load_2d(st_bv(s), &tmv, &full[s], 0, y);
+                    tma_load_2d(st_bv(s) + kBox, &tmv, &full[s], NB == 2 ? 64 : 0, y);
                 }
             }
             for (int s = 0; s < depth; ++s) {                   // drain issued copies
@@ -209,63 +208,29 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     drain_wait(&full[s], (uint32_t)((fills - 1) & 1));
             }
         }
-    } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
+    } else if (warp == 1 || (warp == 3 && !SB)) {
+        // ---------------------------------------------------------------- MMA issuers
+        // warp 1: QK of every tile; warp 3: PV of every tile.  A thread that polls an
+        // mbarrier stalls until its own MMAs have completed, so one issuer for both
+        // serialised them (QK(t+1), drain, PV(t), drain); two let the waits of one
+        // overlap the MMAs of the other.
         if (lane == 0 && n > 0) {
-            const uint32_t idesc_qk = idesc_bf16(128, HH, 0, 0);
-            const uint32_t idesc_pv = idesc_bf16(128, HH, 1, 0);
-            const uint32_t q0 = smem_u32(qbuf), w0 = smem_u32(wbuf);
-            TileWalk<KT> twq, twp;
-            twq.init(P, g0);
-            twp.init(P, g0);
-            int segq = -1, segp = -1;     // segment counters for the QK and PV streams
-            int prev_bq = -1, prev_bp = -1;
-            // PV(j) for the previous tile; returns false on a failed wait
-            auto issue_pv = [&](int j) -> bool {
-                const int g = g0 + j;
-                twp.advance(P, g);
-                const bool first = twp.b != prev_bp;
-                if (first) { ++segp; prev_bp = twp.b; }
-                const bool last = (j == n - 1) || (P.tile_prefix[twp.b + 1] <= g + 1);
-                if (!mbar_wait(&w_full[j & 1], (uint32_t)((j >> 1) & 1), lim, a.err, abort)) return false;
-                if (first && segp > 0 &&
-                    !mbar_wait(o_free, (uint32_t)((segp - 1) & 1), lim, a.err, abort))
-                    return false;
-                const bool vkeep = a.bcap == 0;         // shared basis: one V stage, kept
-                const int s = vkeep ? 0 : j % kVS;
-                if (!mbar_wait(&v_full[s], vkeep ? 0u : (uint32_t)((j / kVS) & 1), lim, a.err, abort))
-                    return false;
-                tc_fence_after();
-                const uint32_t bv = smem_u32(st_bv(s));
-                const uint32_t wb = w0 + (uint32_t)(j & 1) * kQW;
-#pragma unroll
-                for (int k = 0; k < 128 / 16; ++k) {
-                    mma_ss(tmem + 2u * HH, smem_desc(bv + (uint32_t)k * 2048u, kBox, 1024, kSwizzle128),
-                           smem_desc(wb + (uint32_t)(k >> 2) * (HH * 128u) + (uint32_t)(k & 3) * 32u,
-                                     16, 1024, kSwizzle128),
-                           idesc_pv, (first && k == 0) ? 0u : 1u);
-                }
-                mma_commit(&w_empty[j & 1]);
-                if (!vkeep) mma_commit(&v_empty[s]);
-                if (last) mma_commit(o_done);
-                return true;
-            };
-            for (int i = 0; i <= n && !*abort; ++i) {
-                bool newseg = false;
-                if (i < n) {
+            if (warp == 1) {
+                const uint32_t idesc_qk = idesc_bf16(128, HH, 0, 0);
+                const uint32_t q0 = smem_u32(qbuf);
+                TileWalk<KT> twq;
+                twq.init(P, g0);
+                int segq = -1, prev_bq = -1;
+                for (int i = 0; i < n && !*abort; ++i) {
                     twq.advance(P, g0 + i);
-                    newseg = twq.b != prev_bq;
-                }
-                // At a sequence boundary the previous part's last PV goes first: the
-                // softmax reads that part's O^T before it builds the next q~.
-                const bool pv_first = i >= 1 && (i == n || newseg);
-                if (pv_first && !issue_pv(i - 1)) break;
-                if (i < n) {
-                    if (newseg) {
+                    if (twq.b != prev_bq) {
                         ++segq;
                         prev_bq = twq.b;
                         if (!mbar_wait(&q_ready[segq & 1], (uint32_t)((segq >> 1) & 1), lim, a.err, abort)) break;
                     }
+                    // U buffer i&1 is free once the softmax of tile i-2 has read it
+                    if (i >= 2 && !mbar_wait(&w_full[i & 1], (uint32_t)(((i >> 1) - 1) & 1), lim, a.err, abort))
+                        break;
                     const int s = i % a.ks;
                     if (!mbar_wait(&k_full[s], (uint32_t)((i / a.ks) & 1), lim, a.err, abort)) break;
                     tc_fence_after();
@@ -281,23 +246,55 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     }
                     mma_commit(&u_full[i & 1]);
                 }
-                if (i >= 1 && !pv_first && !issue_pv(i - 1)) break;
+            } else {
+                const uint32_t idesc_pv = idesc_bf16(128, HH, 1, 0);
+                const uint32_t w0 = smem_u32(wbuf);
+                TileWalk<KT> twp;
+                twp.init(P, g0);
+                int segp = -1, prev_bp = -1;
+                for (int j = 0; j < n && !*abort; ++j) {
+                    const int g = g0 + j;
+                    twp.advance(P, g);
+                    const bool first = twp.b != prev_bp;
+                    if (first) { ++segp; prev_bp = twp.b; }
+                    const bool last = (j == n - 1) || (P.tile_prefix[twp.b + 1] <= g + 1);
+                    if (!mbar_wait(&w_full[j & 1], (uint32_t)((j >> 1) & 1), lim, a.err, abort)) break;
+                    if (first && segp > 0 &&
+                        !mbar_wait(o_free, (uint32_t)((segp - 1) & 1), lim, a.err, abort))
+                        break;
+                    const int s = j % kVS;
+                    if (!mbar_wait(&v_full[s], (uint32_t)((j / kVS) & 1), lim, a.err, abort)) break;
+                    tc_fence_after();
+                    const uint32_t bv = smem_u32(st_bv(s));
+                    const uint32_t wb = w0 + (uint32_t)(j & 1) * kQW;
+#pragma unroll
+                    for (int k = 0; k < 128 / 16; ++k) {
+                        mma_ss(tmem + 2u * HH, smem_desc(bv + (uint32_t)k * 2048u, kBox, 1024, kSwizzle128),
+                               smem_desc(wb + (uint32_t)(k >> 2) * (HH * 128u) + (uint32_t)(k & 3) * 32u,
+                                         16, 1024, kSwizzle128),
+                               idesc_pv, (first && k == 0) ? 0u : 1u);
+                    }
+                    mma_commit(&w_empty[j & 1]);
+                    mma_commit(&v_empty[s]);
+                    if (last) mma_commit(o_done);
+                }
             }
-            // every MMA issued has completed before TMEM is released
+            // every MMA either issuer issued has completed before TMEM is released
             mma_commit(fin);
             drain_wait(fin, 0);
         }
-    } else {
+    } else if (warp >= 4) {
         // ---------------------------------------------------------------- softmax
-        const int sw = warp - 3;                 // 0 .. 4*NG-1
+        const int sw = warp - 4;                 // 0 .. 4*NG-1
         const int hg = sw >> 2;                  // head group (16 heads)
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;       // TMEM lane = tile row (key j, rank s)
         const int jl = r / R, sr = r % R;
-        const int stid = threadIdx.x - 96;       // 0 .. NSM-1
+        const int stid = threadIdx.x - 128;      // 0 .. NSM-1
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
         const int hbase = hg * 16;
         float m[16], lp[16];
+        float acc[16];                           // SB: sum over keys of p a^V (this row's rank)
         TileWalk<KT> tw;
         if (n > 0) tw.init(P, g0);
         int seg = -1, prev_b = -1;
@@ -353,7 +350,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 bar_sync(3, NSM);
                 if (stid == 0) mbar_arrive(&q_ready[seg & 1]);
 #pragma unroll
-                for (int h = 0; h < 16; ++h) { m[h] = -INFINITY; lp[h] = 0.f; }
+                for (int h = 0; h < 16; ++h) { m[h] = -INFINITY; lp[h] = 0.f; acc[h] = 0.f; }
             }
             const int j0 = (g - P.tile_prefix[b]) * KT;
             const int len = P.len[b];
@@ -400,7 +397,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             }
             // first tile of a part, or a score above the reference max: exact tile max
             if (bar_any(1 + hg, 128, first || over)) {
-                float* rd = red + hg * 64;
+                float* rd = red + hg * 192;
 #pragma unroll
                 for (int h = 0; h < 16; ++h) {
                     float v = warp_max(sc[h]);
@@ -417,9 +414,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     resc |= alpha[h] != 1.f;
                     m[h] = mn;
                     lp[h] *= alpha[h];
+                    if constexpr (SB) acc[h] *= alpha[h];
                 }
                 bar_sync(1 + hg, 128);                 // everyone has read the scratch
-                if (!first && __any_sync(0xffffffffu, resc)) {
+                if (!SB && !first && __any_sync(0xffffffffu, resc)) {
                     // O^T columns of this group *= alpha once PV(i-1) has completed
                     if (!bad)
                         bad = !mbar_wait(&w_empty[(i - 1) & 1], (uint32_t)(((i - 1) >> 1) & 1), lim, a.err, abort);
@@ -433,33 +431,43 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     tmem_st_wait();
                 }
             }
-            // p and W^T (row r = K index, columns = heads), bf16 pairs of adjacent rows
-            if (i >= 2 && !bad)
-                bad = !mbar_wait(&w_empty[i & 1], (uint32_t)(((i >> 1) - 1) & 1), lim, a.err, abort);
-            uint8_t* wb = wbuf + (size_t)(i & 1) * kQW;
+            if constexpr (SB) {
+                // shared basis: every value row of rank s is the basis b^V_s, so the
+                // values need only sum_j p a^V_{j,h,s}, kept per thread (its row's rank)
 #pragma unroll
-            for (int h = 0; h < 16; ++h) {
-                const float p = ex2(sc[h] - m[h]);
-                if (sr == 0) lp[h] += p;
-                const float w = valid ? p * av[h] : 0.f;
-                const float wn = __shfl_down_sync(0xffffffffu, w, 1);
-                if ((r & 1) == 0) {
-                    const int hh = hbase + h;
-                    *reinterpret_cast<uint32_t*>(wb + (r >> 6) * (HH * 128u) + sw128_offset(hh, (r & 63) * 2)) =
-                        pack_bf16(w, wn);
+                for (int h = 0; h < 16; ++h) {
+                    const float p = ex2(sc[h] - m[h]);
+                    if (sr == 0) lp[h] += p;
+                    if (valid) acc[h] = fmaf(p, av[h], acc[h]);
                 }
-            }
-            if (hg == 0 && !valid && j0 + jl >= len && a.bcap != 0) {
-                // keys past the sequence: clear their b^V row (once the tile has landed)
-                // so 0 * (cache contents) = 0.  (The kept shared-basis stage holds finite
-                // basis rows and zero fill only, and is read by every tile.)
-                const int sv = i % kVS;
-                if (!bad) bad = !mbar_wait(&v_full[sv], (uint32_t)((i / kVS) & 1), lim, a.err, abort);
-                if (!bad) {
-                    uint4* z0 = reinterpret_cast<uint4*>(st_bv(sv) + r * 128);
-                    uint4* z1 = reinterpret_cast<uint4*>(st_bv(sv) + kBox + r * 128);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) { z0[e] = make_uint4(0, 0, 0, 0); z1[e] = make_uint4(0, 0, 0, 0); }
+            } else {
+                // p and W^T (row r = K index, columns = heads), bf16 pairs of adjacent rows
+                if (i >= 2 && !bad)
+                    bad = !mbar_wait(&w_empty[i & 1], (uint32_t)(((i >> 1) - 1) & 1), lim, a.err, abort);
+                uint8_t* wb = wbuf + (size_t)(i & 1) * kQW;
+    #pragma unroll
+                for (int h = 0; h < 16; ++h) {
+                    const float p = ex2(sc[h] - m[h]);
+                    if (sr == 0) lp[h] += p;
+                    const float w = valid ? p * av[h] : 0.f;
+                    const float wn = __shfl_down_sync(0xffffffffu, w, 1);
+                    if ((r & 1) == 0) {
+                        const int hh = hbase + h;
+                        *reinterpret_cast<uint32_t*>(wb + (r >> 6) * (HH * 128u) + sw128_offset(hh, (r & 63) * 2)) =
+                            pack_bf16(w, wn);
+                    }
+                }
+                if (hg == 0 && !valid && j0 + jl >= len) {
+                    // keys past the sequence: clear their b^V row (once the tile has landed)
+                    // so 0 * (cache contents) = 0
+                    const int sv = i % kVS;
+                    if (!bad) bad = !mbar_wait(&v_full[sv], (uint32_t)((i / kVS) & 1), lim, a.err, abort);
+                    if (!bad) {
+                        uint4* z0 = reinterpret_cast<uint4*>(st_bv(sv) + r * 128);
+                        uint4* z1 = reinterpret_cast<uint4*>(st_bv(sv) + kBox + r * 128);
+    #pragma unroll
+                        for (int e = 0; e < 8; ++e) { z0[e] = make_uint4(0, 0, 0, 0); z1[e] = make_uint4(0, 0, 0, 0); }
+                    }
                 }
             }
             fence_proxy_async_smem();
@@ -469,18 +477,51 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             const bool last = (i == n - 1) || (P.tile_prefix[b + 1] <= g + 1);
             if (last) {
                 // part done: O^T (lane = d row), l per head, written to the workspace
-                if (!bad) bad = !mbar_wait(o_done, (uint32_t)(seg & 1), lim, a.err, abort);
-                tc_fence_after();
-                uint32_t o[16];
-                tmem_ld16(lane_addr + 2u * HH + hbase, o);
-                tmem_ld_wait();
                 const int part = P.first_part[b] + (c - P.c_first[b]);
                 float* wo = a.ws_o + (size_t)part * HH * DH;
-                if (!bad && r < DH) {
+                if constexpr (SB) {
+                    // S_{h,s} = sum_j p a^V_{j,h,s}: rows of rank s are the lanes of parity
+                    // s (R = 2); sum them in the warp, then over the group's 4 warps, and
+                    // O_h = sum_s S_{h,s} b^V_s, one d_h element per thread
+                    float* rs = red + hg * 192 + 64;     // [4 warps][R][16]
 #pragma unroll
-                    for (int h = 0; h < 16; ++h) wo[(size_t)(hbase + h) * DH + r] = __uint_as_float(o[h]);
+                    for (int h = 0; h < 16; ++h) {
+                        float v = acc[h];
+                        v += __shfl_xor_sync(0xffffffffu, v, 2);
+                        v += __shfl_xor_sync(0xffffffffu, v, 4);
+                        v += __shfl_xor_sync(0xffffffffu, v, 8);
+                        v += __shfl_xor_sync(0xffffffffu, v, 16);
+                        if (lane < R) rs[(quarter * R + lane) * 16 + h] = v;
+                    }
+                    bar_sync(1 + hg, 128);
+                    if (!bad && r < DH) {
+                        float bvr[R];
+#pragma unroll
+                        for (int q = 0; q < R; ++q) bvr[q] = __bfloat162float(a.cb_v[q * DH + r]);
+#pragma unroll
+                        for (int h = 0; h < 16; ++h) {
+                            float o = 0.f;
+#pragma unroll
+                            for (int q = 0; q < R; ++q) {
+                                const float S = (rs[q * 16 + h] + rs[(R + q) * 16 + h]) +
+                                                (rs[(2 * R + q) * 16 + h] + rs[(3 * R + q) * 16 + h]);
+                                o = fmaf(S, bvr[q], o);
+                            }
+                            wo[(size_t)(hbase + h) * DH + r] = o;
+                        }
+                    }
+                } else {
+                    if (!bad) bad = !mbar_wait(o_done, (uint32_t)(seg & 1), lim, a.err, abort);
+                    tc_fence_after();
+                    uint32_t o[16];
+                    tmem_ld16(lane_addr + 2u * HH + hbase, o);
+                    tmem_ld_wait();
+                    if (!bad && r < DH) {
+#pragma unroll
+                        for (int h = 0; h < 16; ++h) wo[(size_t)(hbase + h) * DH + r] = __uint_as_float(o[h]);
+                    }
                 }
-                float* rd = red + hg * 64;
+                float* rd = red + hg * 192;
 #pragma unroll
                 for (int h = 0; h < 16; ++h) {
                     const float v = warp_sum(lp[h]);
@@ -493,8 +534,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     a.ws_ml[((size_t)part * HH + hbase + r) * 2 + 1] = l;
                 }
                 bar_sync(1 + hg, 128);
-                tc_fence_before();
-                mbar_arrive(o_free);
+                if constexpr (!SB) {
+                    tc_fence_before();
+                    mbar_arrive(o_free);
+                }
             }
             if (bar_any(4, NSM, bad)) break;
         }
@@ -507,7 +550,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     }
 }
 
-template <int DH, int HH, int R>
+template <int DH, int HH, int R, bool SB>
 cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const DecodePlan& plan,
                      cudaStream_t st) {
     constexpr int KT = 128 / R;
@@ -515,7 +558,9 @@ cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const D
     const uint32_t a_pad = (a.a_bytes + 127u) & ~127u;
     constexpr int NB = DH / 64;
     a.kstage_bytes = ((NB * kBox + 2u * a_pad) + 1023u) & ~1023u;
-    const size_t fixed = 1024 + (size_t)kVS * 2 * kBox + 4u * HH * 256u + (HH / 16) * 64 * sizeof(float) + 32 * 8 + 16;
+    // (SB: no V ring, no W^T buffers)
+    const size_t fixed = 1024 + (SB ? 0 : (size_t)kVS * 2 * kBox) + (SB ? 2u : 4u) * HH * 256u +
+                         (HH / 16) * 192 * sizeof(float) + 32 * 8 + 16;
     a.ks = 4;
     while (a.ks > 2 && fixed + (size_t)a.ks * a.kstage_bytes > 227 * 1024) --a.ks;
     const size_t smem = fixed + (size_t)a.ks * a.kstage_bytes;
@@ -545,10 +590,10 @@ cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const D
         tmak = tmk;     // unused
         tmav = tmk;
     }
-    constexpr int threads = 96 + 32 * 4 * (HH / 16);
-    cudaError_t e = allow_smem(reinterpret_cast<const void*>(decode_tc_kernel<DH, HH, R>), (int)smem);
+    constexpr int threads = 128 + 32 * 4 * (HH / 16);
+    cudaError_t e = allow_smem(reinterpret_cast<const void*>(decode_tc_kernel<DH, HH, R, SB>), (int)smem);
     if (e != cudaSuccess) return e;
-    decode_tc_kernel<DH, HH, R><<<plan.n_ctas, threads, smem, st>>>(tmk, tmv, tmak, tmav, a, plan);
+    decode_tc_kernel<DH, HH, R, SB><<<plan.n_ctas, threads, smem, st>>>(tmk, tmv, tmak, tmav, a, plan);
     return cudaGetLastError();
 }
 }  // namespace
@@ -576,9 +621,17 @@ cudaError_t launch_decode_tc(const Shape& s, const void* q_a, const void* q_b, c
     a.qscale = 1.4426950408889634f / ((s.Rq > 0 ? (float)s.Rq : 1.f) * (float)s.Rk * std::sqrt((float)s.Dh));
     a.err = err;
     a.wait_limit = wait_limit;
-    if (s.Dh == 64) return s.H == 16 ? launch_t<64, 16, 2>(s, a, c, plan, st)
-                                     : launch_t<64, 32, 2>(s, a, c, plan, st);
-    return s.H == 16 ? launch_t<128, 16, 2>(s, a, c, plan, st) : launch_t<128, 32, 2>(s, a, c, plan, st);
+    a.cb_v = static_cast<const __nv_bfloat16*>(c.b_v);
+    if (s.shared) {
+        if (s.Dh == 64) return s.H == 16 ? launch_t<64, 16, 2, true>(s, a, c, plan, st)
+                                         : launch_t<64, 32, 2, true>(s, a, c, plan, st);
+        return s.H == 16 ? launch_t<128, 16, 2, true>(s, a, c, plan, st)
+                         : launch_t<128, 32, 2, true>(s, a, c, plan, st);
+    }
+    if (s.Dh == 64) return s.H == 16 ? launch_t<64, 16, 2, false>(s, a, c, plan, st)
+                                     : launch_t<64, 32, 2, false>(s, a, c, plan, st);
+    return s.H == 16 ? launch_t<128, 16, 2, false>(s, a, c, plan, st)
+                     : launch_t<128, 32, 2, false>(s, a, c, plan, st);
 }
 
 }  // namespace tpa
