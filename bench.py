@@ -47,10 +47,7 @@ FLUSH_BYTES = 256 << 20          # > 126 MB L2
 # the kernel as it stands (dram__bytes_read.sum + dram__bytes_write.sum); None where no
 # capture of the current kernel exists.  The 32K decode was captured on 16 of its 64
 # sequences and scaled by the keys processed (traffic grows in proportion).
-PROFILED_TRAFFIC = {
-    ("prefill_b8_s2048_d1024", "tpa_prefill"): 26.45e6 + 0.084e6,
-    ("decode_b64_ctx32k", "tpa_decode"): 4 * (604.10e6 + 5.88e6),
-}
+PROFILED_TRAFFIC = {}
 
 
 # ------------------------------------------------------------------ accounting
@@ -530,10 +527,18 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode-leg", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time direct calls instead of graph replays")
+    ap.add_argument("--capture", action="store_true",
+                    help="for an ncu capture: run --warmup untimed steps and one more, print no bench line")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="with --capture: the first N sequences of the workload (a capture-sized case)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.batch and not args.capture:
+        ap.error("--batch only sizes --capture runs")
     wl = I.WORKLOADS[args.workload]
+    if args.batch:
+        wl = I.custom(wl.name, wl, batch=min(args.batch, wl.batch))
 
     if args.impl == "reference":
         ws = int(os.environ.get("WORLD_SIZE", "1"))
@@ -546,6 +551,15 @@ def main():
     pk = peaks()
 
     step = PrefillStep(wl, tpa) if wl.kind == "prefill" else DecodeStep(wl, tpa)
+    if args.capture:
+        # direct calls (no graph, no events), so that ncu -k/-s/-c select launches plainly
+        for _ in range(args.warmup + 1):
+            step.run()
+        torch.cuda.synchronize()
+        assert tpa.tpa_get_device_error() == 0
+        if rank == 0:
+            print(f"captured workload {wl.name}: {args.warmup + 1} steps of {step.launches_per_step} launches")
+        return
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if wl.kind == "prefill" else None
     with ClockSampler(local) as clk:
         ms = timed(step, args.steps, args.warmup, ws, flush, graph=not args.no_graph)
