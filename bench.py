@@ -46,8 +46,14 @@ FLUSH_BYTES = 256 << 20          # > 126 MB L2
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture of
 # the kernel as it stands (dram__bytes_read.sum + dram__bytes_write.sum); None where no
 # capture of the current kernel exists.  The 32K decode was captured on 16 of its 64
-# sequences and scaled by the keys processed (traffic grows in proportion).
-PROFILED_TRAFFIC = {}
+# sequences and the KV-only decode on 4 of its 16, each scaled by the keys processed
+# (traffic grows in proportion); the prefill and the shared-basis decode at full size.
+PROFILED_TRAFFIC = {
+    ("prefill_b8_s2048_d1024", "tpa_prefill"): 26.450e6 + 0.042e6,
+    ("decode_b64_ctx32k", "tpa_decode"): 4 * (604.106e6 + 5.294e6),
+    ("kvonly_decode_b16_ctx64k_128k", "tpa_decode"): 1602374 / 428112 * (548.137e6 + 7.127e6),
+    ("shared_basis_decode_b64_ctx32k", "tpa_decode"): 285.554e6 + 5.801e6,
+}
 
 
 # ------------------------------------------------------------------ accounting
