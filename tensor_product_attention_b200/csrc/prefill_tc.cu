@@ -481,20 +481,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 tc_fence_after();
                 issue_qk(1, 1);
             }
-            // Steady state: one wait for W(t), then PV(t) and QK(t+2) back to back.
-            // QK(t+2) overwrites U_{bl, t&1} after PV(t) has read W from it (one issuer,
-            // in order).  s0 = stage of tile t; s2, ph2 = stage and parity of tile t+2.
+            // Steady state: wait for the stage of tile t+2 (this also drains PV(t-1) and
+            // QK(t+1), while the softmax still works on t), then for W(t), then PV(t) and
+            // QK(t+2) back to back.  QK(t+2) overwrites U_{bl, t&1} after PV(t) has read
+            // W from it (one issuer, in order).  s0 = stage of tile t; s2, ph2 = stage
+            // and parity of tile t+2.
             int s0 = 0, s2 = 2;
             uint32_t ph2 = 0;
             for (int t = 0; ok && t < n_tiles; ++t) {
+                const bool next = t + 2 < n_tiles;
+                if (next && !mbar_wait(&kv_full[s2], ph2, lim, a.err, abort)) break;
                 if (!mbar_wait(&w_ready[2 * bl + (t & 1)], (uint32_t)((t >> 1) & 1), lim, a.err, abort)) break;
                 // block 0's softmax clears the b^V rows past the valid keys of the last
                 // tile before it hands over its W; block 1's PV reads the same stage
                 if (bl == 1 && t == n_tiles - 1 && t * KT + KT > kv_len &&
                     !mbar_wait(&w_ready[t & 1], (uint32_t)((t >> 1) & 1), lim, a.err, abort))
                     break;
-                const bool next = t + 2 < n_tiles;
-                if (next && !mbar_wait(&kv_full[s2], ph2, lim, a.err, abort)) break;
                 tc_fence_after();
                 // O_bl += W_bl(t) . b^V(t)
                 const uint32_t bv = smem_u32(stage_bv(s0));
