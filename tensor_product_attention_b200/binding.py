@@ -8,6 +8,7 @@ All arithmetic runs in the library's CUDA kernels.  Importing this module fails 
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from dataclasses import dataclass
@@ -15,6 +16,9 @@ from dataclasses import dataclass
 import torch
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtpa.so")
+# The bounds-checked build of the same sources (python -m tensor_product_attention_b200.build
+# --debug): a bad index records TPA_DEVERR_BOUNDS (2) in the device error word.
+DEBUG_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtpa_debug.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: run `python -m tensor_product_attention_b200.build`")
 _lib = ctypes.CDLL(LIB_PATH)
@@ -84,10 +88,29 @@ _sig = {
     "tpa_get_device_error": (ctypes.c_int, [ctypes.c_void_p, _i32p]),
     "tpa_set_wait_limit": (None, [ctypes.c_uint32]),
 }
-for _name, (_res, _args) in _sig.items():
-    _fn = getattr(_lib, _name)
-    _fn.restype = _res
-    _fn.argtypes = _args
+def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
+    for name, (res, args) in _sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_declare(_lib)
+
+
+@contextlib.contextmanager
+def use_library(path: str):
+    """Route every call of this module to the library at ``path`` (same ABI) for the
+    duration of the block, e.g. DEBUG_LIB_PATH.  Not thread-safe."""
+    global _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing")
+    prev, _lib = _lib, _declare(ctypes.CDLL(path))
+    try:
+        yield
+    finally:
+        _lib = prev
 
 
 class TPAError(RuntimeError):

@@ -98,6 +98,8 @@ struct DecodeArgs {
     float* ws_o;    // [parts][H][Dh]
     int H, Dh, Rq, Rk, Rv, cap, split_len;
     long long bcap;   // B_K / B_V rows between sequences: cap, or 0 (shared basis)
+    int cache_batch;  // sequences the cache holds (bounds checks)
+    int* err;
 };
 
 template <typename T>
@@ -107,6 +109,9 @@ __global__ void __launch_bounds__(NT) decode_simt_kernel(DecodeArgs a, const Dec
     const int j0 = split * a.split_len;
     if (j0 >= L) return;
     const int j1 = min(L, j0 + a.split_len);
+    // every cache row this CTA reads is (b, j < L); its part slot must exist
+    if (!in_bounds(b < a.cache_batch && L <= a.cap && plan.first_part[b] + split < plan.total_parts, a.err))
+        return;
     const int H = a.H, Dh = a.Dh;
     const int bk_row = a.Rk * Dh + 1;   // padded per-key stride: conflict-free score loop
 
@@ -234,6 +239,7 @@ struct CombineArgs {
     const float* ws_o;
     void* out;
     int H, Dh, Rv;
+    int* err;
 };
 
 // grid (H, batch), one thread per output element of the head.  Parts are merged in
@@ -243,6 +249,7 @@ __global__ void decode_combine_kernel(CombineArgs a, const DecodePlan plan) {
     const int h = blockIdx.x, b = blockIdx.y;
     const int nsplit = plan.n_parts[b];
     const long long base = plan.first_part[b];
+    if (!in_bounds(base >= 0 && base + nsplit <= plan.total_parts, a.err)) return;
     float m = -INFINITY;
     for (int k = 0; k < nsplit; ++k) m = fmaxf(m, a.ws_ml[((base + k) * a.H + h) * 2]);
     float den = 0.f;
@@ -271,10 +278,12 @@ static size_t decode_simt_smem(const Shape& s) {
 }
 
 cudaError_t launch_decode_simt(const Shape& s, const void* q_a, const void* q_b,
-                               const tpa_cache& c, const DecodePlan& plan, float* ws,
+                               const tpa_cache& c, const DecodePlan& plan, float* ws, int* err,
                                cudaStream_t st) {
     if ((long long)s.H * s.Dh > (long long)NT * MAXO) return cudaErrorInvalidValue;
     DecodeArgs a;
+    a.cache_batch = c.batch;
+    a.err = err;
     a.q_a = q_a; a.q_b = q_b;
     a.ca_k = c.a_k; a.ca_v = c.a_v; a.cb_k = c.b_k; a.cb_v = c.b_v;
     a.ws_ml = ws;
@@ -299,8 +308,9 @@ cudaError_t launch_decode_simt(const Shape& s, const void* q_a, const void* q_b,
 }
 
 cudaError_t launch_decode_combine(const Shape& s, const DecodePlan& plan, const float* ws,
-                                  void* out, cudaStream_t st) {
+                                  void* out, int* err, cudaStream_t st) {
     CombineArgs a;
+    a.err = err;
     a.ws_ml = ws;
     a.ws_o = ws + (size_t)plan.total_parts * s.H * 2;
     a.out = out;

@@ -62,6 +62,7 @@ struct DecodeTcArgs {
     float qscale;
     uint32_t a_bytes, kstage_bytes;  // a^K (or a^V) tile; one K-ring stage (b^K, a^K, a^V)
     int ks;                          // K ring depth (2..4, as shared memory allows)
+    int cache_batch;                 // sequences the cache holds (bounds checks)
     int* err;
     uint32_t wait_limit;
 };
@@ -176,6 +177,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     !mbar_wait(&empty[s], (uint32_t)((i / depth - 1) & 1), lim, a.err, abort))
                     break;
                 const int y = (int)(((long long)b * a.bcap + j0) * R);
+                if (kside && !in_bounds(b < a.cache_batch && j0 < a.cap, a.err)) { *abort = 1; break; }
                 if (kside) {
                     // a^K, a^V: one TMA box each, 128-byte rows (one key at h 32, two at
                     // h 16) with the 128-byte swizzle; keys past the tensor read as zeros,
@@ -478,7 +480,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             if (last) {
                 // part done: O^T (lane = d row), l per head, written to the workspace
                 const int part = P.first_part[b] + (c - P.c_first[b]);
-                float* wo = a.ws_o + (size_t)part * HH * DH;
+                if (!in_bounds(part >= 0 && part < P.total_parts, a.err)) bad = true;
+                float* wo = a.ws_o + (size_t)(bad ? 0 : part) * HH * DH;
                 if constexpr (SB) {
                     // S_{h,s} = sum_j p a^V_{j,h,s}: rows of rank s are the lanes of parity
                     // s (R = 2); sum them in the warp, then over the group's 4 warps, and
@@ -618,6 +621,7 @@ cudaError_t launch_decode_tc(const Shape& s, const void* q_a, const void* q_b, c
     a.Rq = s.Rq;
     a.cap = c.capacity;
     a.bcap = (int)b_seq_rows(s, c);
+    a.cache_batch = c.batch;
     a.qscale = 1.4426950408889634f / ((s.Rq > 0 ? (float)s.Rq : 1.f) * (float)s.Rk * std::sqrt((float)s.Dh));
     a.err = err;
     a.wait_limit = wait_limit;

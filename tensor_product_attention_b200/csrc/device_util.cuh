@@ -35,4 +35,19 @@ __device__ __forceinline__ void raise_error(int* err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
 
+// Index checks of the bounds-checked build (-DTPA_DEBUG_BOUNDS, libtpa_debug.so): a
+// plain global access is made only if in_bounds() holds; a failed check records
+// TPA_DEVERR_BOUNDS (2) in the error word and the access is skipped, so a bad index
+// shows up as an error code, never as a fault.  Release builds compile the checks away.
+__device__ __forceinline__ bool in_bounds(bool ok, int* err) {
+#ifdef TPA_DEBUG_BOUNDS
+    if (!ok) raise_error(err, 2);
+    return ok;
+#else
+    (void)ok;
+    (void)err;
+    return true;
+#endif
+}
+
 }  // namespace tpa

@@ -21,6 +21,8 @@ struct PrefillArgs {
     void* out;
     int T, S, H, Dh, Rq, Rk, Rv, cap;
     long long bcap;       // B_K / B_V rows between sequences: cap, or 0 (shared basis)
+    int cache_batch;      // sequences the cache holds (bounds checks)
+    int* err;
 };
 
 template <typename T>
@@ -31,6 +33,8 @@ __global__ void __launch_bounds__(128) prefill_simt_kernel(PrefillArgs a, SeqPar
     const int t = (int)(warp / a.H), h = (int)(warp % a.H);
     const int b = t / a.S, i = t - b * a.S;
     const int pos = start.v[b] + i;
+    // every cache row this warp reads is (b, j <= pos)
+    if (!in_bounds(b < a.cache_batch && pos < a.cap, a.err)) return;
     const T* aq = reinterpret_cast<const T*>(a.a_q);
     const T* bq = reinterpret_cast<const T*>(a.b_q);
     const T* ak = reinterpret_cast<const T*>(a.ca_k);
@@ -98,8 +102,10 @@ __global__ void __launch_bounds__(128) prefill_simt_kernel(PrefillArgs a, SeqPar
 
 cudaError_t launch_prefill_simt(const Shape& s, const tpa_factors& q, const tpa_cache& c,
                                 int batch, int seqlen, const SeqParams& start, void* out,
-                                cudaStream_t st) {
+                                int* err, cudaStream_t st) {
     PrefillArgs a;
+    a.cache_batch = c.batch;
+    a.err = err;
     a.a_q = q.a_q; a.b_q = q.b_q;
     a.ca_k = c.a_k; a.ca_v = c.a_v; a.cb_k = c.b_k; a.cb_v = c.b_v;
     a.out = out;

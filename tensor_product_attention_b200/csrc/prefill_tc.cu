@@ -63,6 +63,8 @@ struct PrefillTcArgs {
     __nv_bfloat16* out;           // [T][H][DH]
     int S, H, Rq, cap, n_qblocks, qpb, stages;
     int bcap;                     // B_K / B_V rows between sequences: cap, or 0 (shared basis)
+    int cache_batch;              // sequences the cache holds (bounds checks)
+    long long T;                  // query rows (bounds checks)
     uint32_t a_bytes;             // bytes of one a^K (or a^V) tile: KT*H*R*2
     uint32_t stage_bytes;
     float qscale, out_scale;
@@ -361,7 +363,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     if (warp >= 4) {
         const int row = threadIdx.x - 128;                // 0..255
         const int i_loc = row / H, h = row - (row / H) * H;
-        const bool vq = i_loc < nq;
+        const bool vq = i_loc < nq && in_bounds((long long)b * a.S + q0 + i_loc < a.T, a.err);
         const long long t = (long long)b * a.S + q0 + (vq ? i_loc : 0);
         // q~ = qscale * sum_r a^Q_r b^Q_r; TPA-KVonly (Rq = 0): qscale * q[t][h][:]
         const int nr = a.Rq > 0 ? a.Rq : 1;
@@ -420,6 +422,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     break;
                 const int j0 = t * KT;
                 const int rows_a = min(KT, a.cap - j0);
+                // the a-factor bulk copies read rows (b, j0 .. j0+rows_a) of the cache
+                if (!in_bounds(b < a.cache_batch && rows_a > 0, a.err)) { *abort = 1; break; }
                 const uint32_t abytes = (uint32_t)rows_a * H * R * 2u;
                 mbar_arrive_expect_tx(&kv_full[s], full_bytes + 2u * abytes);
                 const int yb = b * a.bcap + j0;             // B row of key j0
@@ -809,6 +813,8 @@ cudaError_t launch_prefill_tc(const Shape& s, const tpa_factors& q, const tpa_ca
     a.Rq = s.Rq;
     a.cap = c.capacity;
     a.bcap = (int)b_seq_rows(s, c);
+    a.cache_batch = c.batch;
+    a.T = (long long)batch * seqlen;
     a.qpb = 256 / s.H;
     a.n_qblocks = (seqlen + a.qpb - 1) / a.qpb;
     a.qscale = 1.4426950408889634f / ((float)(s.Rq > 0 ? s.Rq : 1) * (float)s.Rk * std::sqrt((float)s.Dh));

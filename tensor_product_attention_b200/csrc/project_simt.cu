@@ -19,6 +19,7 @@ struct ProjArgs {
     int T, N, D, seqlen, Dh;
     const float2* cs;
     ProjLayout L;
+    int* err;
 };
 
 __device__ __forceinline__ int segment_of(const ProjLayout& L, int c) {
@@ -29,10 +30,13 @@ __device__ __forceinline__ int segment_of(const ProjLayout& L, int c) {
 }
 
 template <typename T>
-__device__ __forceinline__ void store_col(const ProjLayout& L, int seg, int t, long long tkv, int c, float v) {
+__device__ __forceinline__ void store_col(const ProjLayout& L, int seg, int t, long long tkv, int c, float v,
+                                          int* err) {
     int width = L.off[seg + 1] - L.off[seg];
     T* dst = reinterpret_cast<T*>(L.dst[seg]);
-    dst[seg_row(L, seg, t, tkv) * width + (c - L.off[seg])] = from_f<T>(v);
+    const long long row = seg_row(L, seg, t, tkv);
+    if (in_bounds(row >= 0 && row < L.rows[seg] && c - L.off[seg] < width, err))
+        dst[row * width + (c - L.off[seg])] = from_f<T>(v);
 }
 
 template <typename T>
@@ -78,7 +82,9 @@ __global__ void __launch_bounds__(NT) project_simt_kernel(ProjArgs a, SeqParams 
         int pos = start.v[b] + (t - b * a.seqlen);
         const long long tkv = (long long)b * L.kv_cap + pos;
         // cache mode: the sequence's last token records the new length, once
-        if (L.lengths && col0 == 0 && tx == 0 && t - b * a.seqlen == a.seqlen - 1) L.lengths[b] = pos + 1;
+        if (L.lengths && col0 == 0 && tx == 0 && t - b * a.seqlen == a.seqlen - 1 &&
+            in_bounds(b < L.n_lengths, a.err))
+            L.lengths[b] = pos + 1;
 #pragma unroll
         for (int jp = 0; jp < 2; ++jp) {
             int c = col0 + tx * 4 + 2 * jp;
@@ -89,12 +95,13 @@ __global__ void __launch_bounds__(NT) project_simt_kernel(ProjArgs a, SeqParams 
                 // segment starts are even, so (c, c+1) is one RoPE pair (2k, 2k+1)
                 int local = c - L.off[seg];
                 int k2 = (local % a.Dh) >> 1;
-                float2 r = a.cs[(long long)pos * (a.Dh >> 1) + k2];
-                store_col<T>(L, seg, t, tkv, c, y0 * r.x - y1 * r.y);
-                store_col<T>(L, seg, t, tkv, c + 1, y0 * r.y + y1 * r.x);
+                float2 r = make_float2(1.f, 0.f);
+                if (in_bounds(pos < L.cs_rows, a.err)) r = a.cs[(long long)pos * (a.Dh >> 1) + k2];
+                store_col<T>(L, seg, t, tkv, c, y0 * r.x - y1 * r.y, a.err);
+                store_col<T>(L, seg, t, tkv, c + 1, y0 * r.y + y1 * r.x, a.err);
             } else {
-                store_col<T>(L, seg, t, tkv, c, y0);
-                if (c + 1 < a.N) store_col<T>(L, segment_of(L, c + 1), t, tkv, c + 1, y1);
+                store_col<T>(L, seg, t, tkv, c, y0, a.err);
+                if (c + 1 < a.N) store_col<T>(L, segment_of(L, c + 1), t, tkv, c + 1, y1, a.err);
             }
         }
     }
@@ -103,8 +110,9 @@ __global__ void __launch_bounds__(NT) project_simt_kernel(ProjArgs a, SeqParams 
 
 cudaError_t launch_project_simt(const Shape& s, const void* x, const void* w, int batch,
                                 int seqlen, const SeqParams& start, const float* cs,
-                                const ProjLayout& L, cudaStream_t st) {
+                                const ProjLayout& L, int* err, cudaStream_t st) {
     ProjArgs a;
+    a.err = err;
     a.x = x; a.w = w; a.T = batch * seqlen; a.N = L.off[6]; a.D = s.D; a.seqlen = seqlen;
     a.Dh = s.Dh; a.cs = reinterpret_cast<const float2*>(cs); a.L = L;
     dim3 grid((a.N + BN - 1) / BN, (a.T + BM - 1) / BM);

@@ -47,12 +47,14 @@ __device__ __forceinline__ int seg_of(const ProjLayout& L, int c) {
 // Store output columns [c0, min(c0+16, N)) of token t (v already rotated); tkv is the
 // token's cache row (cache mode).
 __device__ __forceinline__ void store16(const ProjLayout& L, int N, long long t, long long tkv, int c0,
-                                        const float (&v)[16]) {
+                                        const float (&v)[16], int* err) {
     const int s0 = seg_of(L, c0);
     const int last = min(c0 + 15, N - 1);
     if (c0 + 15 < N && seg_of(L, last) == s0) {
         const int width = L.off[s0 + 1] - L.off[s0];
-        const long long e = seg_row(L, s0, t, tkv) * width + (c0 - L.off[s0]);
+        const long long row = seg_row(L, s0, t, tkv);
+        if (!in_bounds(row >= 0 && row < L.rows[s0], err)) return;
+        const long long e = row * width + (c0 - L.off[s0]);
         __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(L.dst[s0]) + e;
         if ((e & 7) == 0) {
             uint4 w0, w1;
@@ -71,8 +73,9 @@ __device__ __forceinline__ void store16(const ProjLayout& L, int N, long long t,
         if (c < N) {
             const int s = seg_of(L, c);
             const int width = L.off[s + 1] - L.off[s];
-            reinterpret_cast<__nv_bfloat16*>(L.dst[s])[seg_row(L, s, t, tkv) * width + (c - L.off[s])] =
-                __float2bfloat16_rn(v[j]);
+            const long long row = seg_row(L, s, t, tkv);
+            if (in_bounds(row >= 0 && row < L.rows[s], err))
+                reinterpret_cast<__nv_bfloat16*>(L.dst[s])[row * width + (c - L.off[s])] = __float2bfloat16_rn(v[j]);
         }
     }
 }
@@ -195,7 +198,9 @@ project_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
                 pos = start.v[b] + i;
                 tkv = (long long)b * a.L.kv_cap + pos;
                 // cache mode: the sequence's last token records the new length, once
-                if (a.L.lengths && n == 0 && colhalf == 0 && i == a.seqlen - 1) a.L.lengths[b] = pos + 1;
+                if (a.L.lengths && n == 0 && colhalf == 0 && i == a.seqlen - 1 &&
+                    in_bounds(b < a.L.n_lengths, a.err))
+                    a.L.lengths[b] = pos + 1;
             }
             const int col0 = n * a.BN;
             const int cend = min(a.N, col0 + a.BN);
@@ -208,7 +213,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
                     const int cc = cg + 2 * j;
                     const int sg = seg_of(a.L, cc);
                     rot[j] = make_float2(1.f, 0.f);
-                    if (valid && (sg == 3 || sg == 4) && cc < cend) {
+                    if (valid && (sg == 3 || sg == 4) && cc < cend && in_bounds(pos < a.L.cs_rows, a.err)) {
                         const int kp = ((cc - a.L.off[sg]) % a.Dh) >> 1;
                         rot[j] = __ldg(&a.cs[(long long)pos * half + kp]);
                     }
@@ -224,8 +229,8 @@ project_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
                     v[2 * j] = x0 * rot[j].x - x1 * rot[j].y;
                     v[2 * j + 1] = x0 * rot[j].y + x1 * rot[j].x;
                 }
-                store16(a.L, cend, t, tkv, cg, *reinterpret_cast<float(*)[16]>(&v[0]));
-                if (cg + 16 < cend) store16(a.L, cend, t, tkv, cg + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+                store16(a.L, cend, t, tkv, cg, *reinterpret_cast<float(*)[16]>(&v[0]), a.err);
+                if (cg + 16 < cend) store16(a.L, cend, t, tkv, cg + 16, *reinterpret_cast<float(*)[16]>(&v[16]), a.err);
             }
             tc_fence_before();
             __syncwarp();

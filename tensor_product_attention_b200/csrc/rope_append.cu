@@ -48,6 +48,9 @@ struct AppendArgs {
     long long row_units[4];   // units of V per token row
     int batch, n_tokens, capacity;
     int32_t* lengths;
+    long long dst_rows;      // cache rows (batch * capacity): bounds checks
+    int n_lengths;
+    int* err;
 };
 
 // grid.y selects one of the four cached tensors; grid.x strides over its rows.
@@ -55,7 +58,7 @@ template <typename V>
 __global__ void append_kernel(AppendArgs a, SeqParams start) {
     if (blockIdx.x == 0 && blockIdx.y == 0) {
         for (int b = threadIdx.x; b < a.batch; b += blockDim.x)
-            a.lengths[b] = start.v[b] + a.n_tokens;
+            if (in_bounds(b < a.n_lengths, a.err)) a.lengths[b] = start.v[b] + a.n_tokens;
     }
     const int arr = blockIdx.y;
     const long long ru = a.row_units[arr];
@@ -69,12 +72,12 @@ __global__ void append_kernel(AppendArgs a, SeqParams start) {
         int b = (int)(tok / a.n_tokens);
         int i = (int)(tok - (long long)b * a.n_tokens);
         long long row = (long long)b * a.capacity + start.v[b] + i;
-        dst[row * ru + e] = src[u];
+        if (in_bounds(row < a.dst_rows && start.v[b] + i < a.capacity, a.err)) dst[row * ru + e] = src[u];
     }
 }
 
 cudaError_t launch_cache_append(const Shape& s, const tpa_cache& c, const tpa_factors& kv,
-                                int batch, int n_tokens, const SeqParams& start,
+                                int batch, int n_tokens, const SeqParams& start, int* err,
                                 cudaStream_t st) {
     const int es = s.bf16 ? 2 : 4;
     const int n_arr = s.shared ? 2 : 4;       // shared basis: A_K, A_V only
@@ -91,6 +94,7 @@ cudaError_t launch_cache_append(const Shape& s, const tpa_cache& c, const tpa_fa
     a.dst[2] = (char*)c.b_k; a.dst[3] = (char*)c.b_v;
     for (int i = 0; i < 4; ++i) a.row_units[i] = row_bytes[i] / vec;
     a.batch = batch; a.n_tokens = n_tokens; a.capacity = c.capacity; a.lengths = c.lengths;
+    a.dst_rows = (long long)c.batch * c.capacity; a.n_lengths = c.batch; a.err = err;
     long long most = 0;
     for (int i = 0; i < n_arr; ++i) {
         long long t = (long long)batch * n_tokens * a.row_units[i];

@@ -85,7 +85,7 @@ tpa_status run_project(const Shape& s, const void* x, const void* w, int batch, 
     if (s.bf16 && project_tc_supported(s, batch * seqlen))
         return launched(launch_project_tc(s, x, w, batch, seqlen, sp, rope_cs, L,
                                           device_error_ptr(), wait_limit(), cs));
-    return launched(launch_project_simt(s, x, w, batch, seqlen, sp, rope_cs, L, cs));
+    return launched(launch_project_simt(s, x, w, batch, seqlen, sp, rope_cs, L, device_error_ptr(), cs));
 }
 
 // Split-K decode and the fixed-order merge of its parts (validated arguments).
@@ -99,9 +99,9 @@ tpa_status run_decode(const Shape& s, const void* q_a, const void* q_b, const tp
     if (decode_workspace_bytes(s, plan) > workspace_bytes) return TPA_ERR_WORKSPACE;
     float* ws = static_cast<float*>(workspace);
     cudaError_t e = tc ? launch_decode_tc(s, q_a, q_b, c, plan, ws, device_error_ptr(), wait_limit(), cs)
-                       : launch_decode_simt(s, q_a, q_b, c, plan, ws, cs);
+                       : launch_decode_simt(s, q_a, q_b, c, plan, ws, device_error_ptr(), cs);
     if (e != cudaSuccess) return TPA_ERR_CUDA;
-    return launched(launch_decode_combine(s, plan, ws, out, cs));
+    return launched(launch_decode_combine(s, plan, ws, out, device_error_ptr(), cs));
 }
 
 }  // namespace
@@ -111,8 +111,13 @@ extern "C" {
 int32_t tpa_abi_version(void) { return TPA_ABI_VERSION; }
 
 const char* tpa_build_info(void) {
+#ifdef TPA_DEBUG_BOUNDS
+    return "libtpa: TPA hot path for sm_100a (tcgen05/TMA kernels for bf16, CUDA-core "
+           "kernels for fp32), bounds-checked build";
+#else
     return "libtpa: TPA hot path for sm_100a (tcgen05/TMA kernels for bf16, CUDA-core "
            "kernels for fp32)";
+#endif
 }
 
 const char* tpa_status_string(tpa_status s) {
@@ -169,8 +174,8 @@ tpa_status tpa_project(const tpa_dims* d, const void* x, const void* w_cat, int3
         sp.v[b] = start_pos[b];
     }
     Shape s = shape_of(*d);
-    return run_project(s, x, w_cat, batch, seqlen, sp, rope_cs, proj_layout(s, *out),
-                       (cudaStream_t)stream);
+    return run_project(s, x, w_cat, batch, seqlen, sp, rope_cs,
+                       proj_layout(s, *out, (long long)batch * seqlen, max_pos), (cudaStream_t)stream);
 }
 
 tpa_status tpa_cache_append(const tpa_dims* d, const tpa_cache* c, const tpa_factors* kv,
@@ -192,7 +197,7 @@ tpa_status tpa_cache_append(const tpa_dims* d, const tpa_cache* c, const tpa_fac
         sp.v[b] = start_pos[b];
     }
     return launched(launch_cache_append(shape_of(*d), *c, *kv, batch, n_tokens, sp,
-                                        (cudaStream_t)stream));
+                                        device_error_ptr(), (cudaStream_t)stream));
 }
 
 tpa_status tpa_shared_basis_tables(const tpa_dims* d, const void* basis_k, const void* basis_v,
@@ -235,7 +240,7 @@ tpa_status tpa_prefill(const tpa_dims* d, const tpa_factors* q, const tpa_cache*
     if (s.bf16 && prefill_tc_supported(s))
         return launched(launch_prefill_tc(s, *q, *c, batch, seqlen, sp, out,
                                           device_error_ptr(), wait_limit(), cs));
-    return launched(launch_prefill_simt(s, *q, *c, batch, seqlen, sp, out, cs));
+    return launched(launch_prefill_simt(s, *q, *c, batch, seqlen, sp, out, device_error_ptr(), cs));
 }
 
 size_t tpa_decode_workspace_bytes(const tpa_dims* d, const int32_t* lengths, int32_t batch) {
@@ -281,7 +286,7 @@ tpa_status tpa_output_project(const tpa_dims* d, const void* attn, const void* w
     ProjLayout L;
     for (int i = 0; i < 6; ++i) L.off[i] = 0;
     L.off[6] = d->d_model;
-    for (int i = 0; i < 6; ++i) L.dst[i] = out;
+    for (int i = 0; i < 6; ++i) { L.dst[i] = out; L.rows[i] = T; }
     SeqParams sp;
     sp.v[0] = 0;
     return run_project(s, attn, w_o, 1, T, sp, nullptr, L, (cudaStream_t)stream);
@@ -334,9 +339,11 @@ tpa_status tpa_decode_step(const tpa_dims* d, const void* x, const void* w_cat,
     f.a_q = s.Rq > 0 ? wsb : nullptr;
     f.b_q = wsb + aq_bytes;
     f.a_k = c->a_k; f.a_v = c->a_v; f.b_k = c->b_k; f.b_v = c->b_v;
-    ProjLayout L = proj_layout(s, f);
+    ProjLayout L = proj_layout(s, f, batch, max_pos);
     L.kv_cap = c->capacity;
     L.lengths = c->lengths;
+    L.n_lengths = c->batch;
+    for (int i : {1, 2, 4, 5}) L.rows[i] = (long long)c->batch * c->capacity;
     cudaStream_t cs = (cudaStream_t)stream;
     // check the decode half before anything is launched
     {

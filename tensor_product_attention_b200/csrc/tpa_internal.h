@@ -44,6 +44,11 @@ struct ProjLayout {
     // also sets lengths[b] = start[b] + seqlen.  Otherwise every segment is at row t.
     int kv_cap = 0;
     int32_t* lengths = nullptr;
+    // Extents for the bounds-checked build: destination rows of each segment, entries
+    // of `lengths`, rows of the RoPE table.
+    long long rows[6] = {0, 0, 0, 0, 0, 0};
+    int n_lengths = 0;
+    int cs_rows = 0;
 };
 
 // Destination row of segment s for token t (tkv: its cache row in cache mode).
@@ -51,8 +56,10 @@ __host__ __device__ inline long long seg_row(const ProjLayout& L, int s, long lo
     return (L.kv_cap > 0 && s != 0 && s != 3) ? tkv : t;
 }
 
-inline ProjLayout proj_layout(const Shape& s, const tpa_factors& f) {
+inline ProjLayout proj_layout(const Shape& s, const tpa_factors& f, long long T, int cs_rows) {
     ProjLayout L;
+    for (int i = 0; i < 6; ++i) L.rows[i] = T;
+    L.cs_rows = cs_rows;
     const int q_rows = s.Rq > 0 ? s.Rq : s.H;
     int w[6] = {s.H * s.Rq, s.H * s.Rk, s.H * s.Rv, q_rows * s.Dh,
                 s.shared ? 0 : s.Rk * s.Dh, s.shared ? 0 : s.Rv * s.Dh};
@@ -91,7 +98,7 @@ cudaError_t launch_rope_table(float* cs, int max_pos, int head_dim, double base,
 
 cudaError_t launch_project_simt(const Shape& s, const void* x, const void* w, int batch,
                                 int seqlen, const SeqParams& start, const float* cs,
-                                const ProjLayout& L, cudaStream_t st);
+                                const ProjLayout& L, int* err, cudaStream_t st);
 
 cudaError_t launch_project_tc(const Shape& s, const void* x, const void* w, int batch,
                               int seqlen, const SeqParams& start, const float* cs,
@@ -104,12 +111,12 @@ cudaError_t launch_shared_basis_tables(const Shape& s, const void* basis_k, cons
                                        void* table_v, cudaStream_t st);
 
 cudaError_t launch_cache_append(const Shape& s, const tpa_cache& c, const tpa_factors& kv,
-                                int batch, int n_tokens, const SeqParams& start,
+                                int batch, int n_tokens, const SeqParams& start, int* err,
                                 cudaStream_t st);
 
 cudaError_t launch_prefill_simt(const Shape& s, const tpa_factors& q, const tpa_cache& c,
                                 int batch, int seqlen, const SeqParams& start, void* out,
-                                cudaStream_t st);
+                                int* err, cudaStream_t st);
 
 cudaError_t launch_prefill_tc(const Shape& s, const tpa_factors& q, const tpa_cache& c,
                               int batch, int seqlen, const SeqParams& start, void* out,
@@ -117,7 +124,7 @@ cudaError_t launch_prefill_tc(const Shape& s, const tpa_factors& q, const tpa_ca
 bool prefill_tc_supported(const Shape& s);
 
 cudaError_t launch_decode_simt(const Shape& s, const void* q_a, const void* q_b,
-                               const tpa_cache& c, const DecodePlan& plan, float* ws,
+                               const tpa_cache& c, const DecodePlan& plan, float* ws, int* err,
                                cudaStream_t st);
 
 cudaError_t launch_decode_tc(const Shape& s, const void* q_a, const void* q_b,
@@ -126,6 +133,6 @@ cudaError_t launch_decode_tc(const Shape& s, const void* q_a, const void* q_b,
 bool decode_tc_supported(const Shape& s);
 
 cudaError_t launch_decode_combine(const Shape& s, const DecodePlan& plan, const float* ws,
-                                  void* out, cudaStream_t st);
+                                  void* out, int* err, cudaStream_t st);
 
 }  // namespace tpa

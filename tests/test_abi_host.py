@@ -163,3 +163,14 @@ def test_shared_basis_host_validation(bnd):
     cache = bnd.tpa_cache(fake, fake, fake, fake, fake, 1, 8)
     assert bnd._lib.tpa_cache_append(by(d), by(cache), by(f), 1, 1, bnd._ints([0]), None) == 1
     assert bnd._lib.tpa_cache_append(by(d), by(cache), by(f), 1, 1, bnd._ints([8]), None) == 1
+
+
+def test_bounds_checked_library_has_the_same_abi(bnd):
+    """libtpa_debug.so (TPA_DEBUG_BOUNDS) exports every declared symbol and says so."""
+    lib = ctypes.CDLL(bnd.DEBUG_LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    with bnd.use_library(bnd.DEBUG_LIB_PATH):
+        assert "bounds-checked" in bnd.tpa_build_info()
+        assert bnd.tpa_abi_version() == 2
+    assert "bounds-checked" not in bnd.tpa_build_info()
