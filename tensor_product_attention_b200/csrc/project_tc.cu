@@ -245,7 +245,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
     }
 }
 
-int pick_bn(int N) {
+int pick_bn(int N, int T) {
     int best_bn = 256, best_waste = 1 << 30;
     const int nt0 = (N + 255) / 256;
     for (int nt = nt0; nt <= nt0 + 3; ++nt) {
@@ -254,6 +254,14 @@ int pick_bn(int N) {
         if (bn > 256 || bn < 16) continue;
         const int waste = nt * bn - N;
         if (waste < best_waste) { best_waste = waste; best_bn = bn; }
+    }
+    // Few row tiles (small batches, e.g. one decode token per sequence): narrower column
+    // tiles spread the weight stream over more SMs instead of a handful of CTAs.
+    const long long m_tiles = (T + BM - 1) / BM, sms = sm_count();
+    if (m_tiles * ((N + best_bn - 1) / best_bn) < sms) {
+        int bn = (int)((N * m_tiles + sms - 1) / sms);
+        bn = std::max(16, (bn + 15) / 16 * 16);
+        best_bn = std::min(best_bn, bn);
     }
     return best_bn;
 }
@@ -272,7 +280,7 @@ cudaError_t launch_project_tc(const Shape& s, const void* x, const void* w, int 
     a.D = s.D;
     a.seqlen = seqlen;
     a.Dh = s.Dh;
-    a.BN = pick_bn(a.N);
+    a.BN = pick_bn(a.N, a.T);
     a.n_tiles_n = (a.N + a.BN - 1) / a.BN;
     a.n_tiles = ((a.T + BM - 1) / BM) * a.n_tiles_n;
     a.k_blocks = (a.D + BK - 1) / BK;
