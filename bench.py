@@ -52,7 +52,6 @@ PROFILED_TRAFFIC = {
     ("prefill_b8_s2048_d1024", "tpa_prefill"): 26.450e6 + 0.042e6,
     ("decode_b64_ctx32k", "tpa_decode"): 4 * (604.106e6 + 5.294e6),
     ("kvonly_decode_b16_ctx64k_128k", "tpa_decode"): 1602374 / 428112 * (548.137e6 + 7.127e6),
-    ("shared_basis_decode_b64_ctx32k", "tpa_decode"): 285.554e6 + 5.801e6,
 }
 
 

@@ -20,10 +20,55 @@
 
 namespace tpa {
 
+// Paired plan: unit u = sequences (2u, 2u+1) (the last unit of an odd batch has one);
+// its tiles cover the longer member.  The CTAs c_first[u] .. c_first[u] + n - 1 that
+// overlap the unit give member 0 parts base .. base+n-1 and member 1 parts
+// base+n .. base+2n-1, so each sequence's parts stay consecutive for the merge.
+static void make_paired_plan(const int32_t* lengths, int batch, int kt, DecodePlan* plan) {
+    DecodePlan& P = *plan;
+    const int U = (batch + 1) / 2;
+    P.n_units = U;
+    long long n = 0;
+    for (int u = 0; u < U; ++u) {
+        P.tile_prefix[u] = (int32_t)n;
+        const int len = std::max(lengths[2 * u], 2 * u + 1 < batch ? lengths[2 * u + 1] : 0);
+        n += (len + kt - 1) / kt;
+    }
+    P.tile_prefix[U] = (int32_t)n;
+    P.total_tiles = (int32_t)n;
+    const int G = (int)std::min<long long>(sm_count(), n);
+    P.n_ctas = G;
+    int32_t n_cta[TPA_MAX_BATCH];
+    for (int u = 0; u < U; ++u) n_cta[u] = 0;
+    int u = 0;
+    for (int c = 0; c < G; ++c) {
+        const long long lo = c * n / G, hi = (c + 1) * n / G;
+        while (u < U && P.tile_prefix[u + 1] <= lo) ++u;
+        for (int uu = u; uu < U && P.tile_prefix[uu] < hi; ++uu) {
+            if (P.tile_prefix[uu + 1] <= lo) continue;
+            if (n_cta[uu] == 0) P.c_first[uu] = c;
+            ++n_cta[uu];
+        }
+    }
+    int part = 0;
+    for (int v = 0; v < U; ++v) {
+        for (int m = 0; m < 2; ++m) {
+            const int b = 2 * v + m;
+            if (b >= batch) break;
+            P.first_part[b] = part;
+            P.n_parts[b] = n_cta[v];
+            part += n_cta[v];
+        }
+    }
+    P.total_parts = part;
+}
+
 void make_decode_plan(const Shape& s, const int32_t* lengths, int batch, bool tc,
                       DecodePlan* plan) {
     DecodePlan& P = *plan;
     P.batch = batch;
+    P.pairs = 0;
+    P.n_units = batch;
     long long total = 0;
     for (int b = 0; b < batch; ++b) {
         P.len[b] = lengths[b];
@@ -48,10 +93,16 @@ void make_decode_plan(const Shape& s, const int32_t* lengths, int batch, bool tc
         P.total_tiles = 0;
         return;
     }
-    // persistent grid over the concatenated key tiles of all sequences
+    // persistent grid over the concatenated key tiles of all sequences (or units)
     const int kt = 128 / s.Rk;
     P.key_tile = kt;
     P.split_len = 0;
+    P.pairs = decode_pairs(s) ? 1 : 0;
+    if (P.pairs) {
+        make_paired_plan(lengths, batch, kt, &P);
+        return;
+    }
+    P.n_units = batch;
     long long n = 0;
     for (int b = 0; b < batch; ++b) {
         P.tile_prefix[b] = (int32_t)n;

@@ -80,7 +80,7 @@ struct TileWalk {
     }
 };
 
-template <int DH, int HH, int R, bool SB>
+template <int DH, int HH, int R, bool SB, bool PAIR>
 __global__ void __launch_bounds__(128 + 32 * 4 * (HH / 16), 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                  const __grid_constant__ CUtensorMap tmak, const __grid_constant__ CUtensorMap tmav,
@@ -90,6 +90,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     constexpr int NG = HH / 16;                 // head groups of 16 (4 warps each)
     constexpr int NSM = 128 * NG;               // softmax threads
     constexpr uint32_t kQW = HH * 256u;         // q~ or W^T buffer: 2 x [HH rows][128 B]
+    // PAIR (shared basis, h 16): the HH = 32 columns are two sequences' 16 heads; a tile
+    // walks one unit (2u, 2u+1); head group hg serves member hg.
+    static_assert(!PAIR || (SB && HH == 32), "pairs: shared-basis kernel, two sequences of 16 heads");
+    constexpr int HS = PAIR ? HH / 2 : HH;      // heads per sequence
+    constexpr int NM = PAIR ? 2 : 1;            // sequences per tile
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -118,9 +123,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     auto st_bk = [&](int s) { return kring + (size_t)s * a.kstage_bytes; };
-    auto st_ak = [&](int s) { return kring + (size_t)s * a.kstage_bytes + NB * kBox; };
-    auto st_av = [&](int s) {
-        return kring + (size_t)s * a.kstage_bytes + NB * kBox + ((a.a_bytes + 127u) & ~127u);
+    const uint32_t a_pad = (a.a_bytes + 127u) & ~127u;
+    // member m's a^K, a^V tiles follow the b^K box
+    auto st_ak = [&](int s, int m = 0) {
+        return kring + (size_t)s * a.kstage_bytes + NB * kBox + (size_t)(2 * m) * a_pad;
+    };
+    auto st_av = [&](int s, int m = 0) {
+        return kring + (size_t)s * a.kstage_bytes + NB * kBox + (size_t)(2 * m + 1) * a_pad;
     };
     auto st_bv = [&](int s) { return vring + (size_t)s * 2 * kBox; };
 
@@ -177,24 +186,30 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     !mbar_wait(&empty[s], (uint32_t)((i / depth - 1) & 1), lim, a.err, abort))
                     break;
                 const int y = (int)(((long long)b * a.bcap + j0) * R);
-                if (kside && !in_bounds(b < a.cache_batch && j0 < a.cap, a.err)) { *abort = 1; break; }
+                if (kside && !in_bounds(NM * b < a.cache_batch && j0 < a.cap, a.err)) { *abort = 1; break; }
                 if (kside) {
                     // a^K, a^V: one TMA box each, 128-byte rows (one key at h 32, two at
                     // h 16) with the 128-byte swizzle; keys past the tensor read as zeros,
                     // so the box lands whole.  Otherwise (h 16) bulk copies of the valid rows.
+                    // PAIR: both members' tiles (an odd batch's last unit loads member 0
+                    // twice; its second group masks every key).
                     const int rows_a = a.asw ? KT : min(KT, a.cap - j0);
-                    const uint32_t abytes = (uint32_t)rows_a * HH * R * 2u;
-                    mbar_arrive_expect_tx(&full[s], NB * kBox + 2u * abytes);
+                    const uint32_t abytes = (uint32_t)rows_a * HS * R * 2u;
+                    mbar_arrive_expect_tx(&full[s], NB * kBox + 2u * NM * abytes);
                     tma_load_2d(st_bk(s), &tmk, &full[s], 0, y);
                     if (NB == 2) tma_load_2d(st_bk(s) + kBox, &tmk, &full[s], 64, y);
-                    if (a.asw) {
-                        const int ya = (b * a.cap + j0) / (128 / (HH * R * 2));
-                        tma_load_2d(st_ak(s), &tmak, &full[s], 0, ya);
-                        tma_load_2d(st_av(s), &tmav, &full[s], 0, ya);
-                    } else {
-                        const long long ea = ((long long)b * a.cap + j0) * HH * R;
-                        bulk_load(st_ak(s), a.ca_k + ea, abytes, &full[s]);
-                        bulk_load(st_av(s), a.ca_v + ea, abytes, &full[s]);
+#pragma unroll
+                    for (int m = 0; m < NM; ++m) {
+                        const int sq = (NM * b + m < a.cache_batch) ? NM * b + m : NM * b;
+                        if (a.asw) {
+                            const int ya = (sq * a.cap + j0) / (128 / (HS * R * 2));
+                            tma_load_2d(st_ak(s, m), &tmak, &full[s], 0, ya);
+                            tma_load_2d(st_av(s, m), &tmav, &full[s], 0, ya);
+                        } else {
+                            const long long ea = ((long long)sq * a.cap + j0) * HS * R;
+                            bulk_load(st_ak(s, m), a.ca_k + ea, abytes, &full[s]);
+                            bulk_load(st_av(s, m), a.ca_v + ea, abytes, &full[s]);
+                        }
                     }
                 } else {
                     // the value MMA has M = 128 rows of d_h: for d_h = 64 the one box is
@@ -316,13 +331,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 uint8_t* qb = qbuf + (size_t)(seg & 1) * kQW;
                 for (int e = stid; e < HH * (DH / 8); e += NSM) {
                     const int h = e / (DH / 8), k8 = (e % (DH / 8)) * 8;
+                    // column h is head qh of sequence qs (PAIR: member h / HS of the unit)
+                    const int qs = NM * b + h / HS, qh = h % HS;
                     float acc[8];
-                    if (a.Rq > 0) {
 #pragma unroll
-                        for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+                    for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+                    if (qs >= P.batch) {
+                        // an odd batch's last unit: no second sequence (its group masks all keys)
+                    } else if (a.Rq > 0) {
                         for (int rq = 0; rq < a.Rq; ++rq) {
-                            const float aqv = __bfloat162float(a.q_a[((long long)b * HH + h) * a.Rq + rq]);
-                            const uint4 raw = *reinterpret_cast<const uint4*>(a.q_b + ((long long)b * a.Rq + rq) * DH + k8);
+                            const float aqv = __bfloat162float(a.q_a[((long long)qs * HS + qh) * a.Rq + rq]);
+                            const uint4 raw = *reinterpret_cast<const uint4*>(a.q_b + ((long long)qs * a.Rq + rq) * DH + k8);
                             const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
                             for (int x = 0; x < 4; ++x) {
@@ -332,7 +351,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                             }
                         }
                     } else {
-                        const uint4 raw = *reinterpret_cast<const uint4*>(a.q_b + ((long long)b * HH + h) * DH + k8);
+                        const uint4 raw = *reinterpret_cast<const uint4*>(a.q_b + ((long long)qs * HS + qh) * DH + k8);
                         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
                         for (int x = 0; x < 4; ++x) {
@@ -355,7 +374,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 for (int h = 0; h < 16; ++h) { m[h] = -INFINITY; lp[h] = 0.f; acc[h] = 0.f; }
             }
             const int j0 = (g - P.tile_prefix[b]) * KT;
-            const int len = P.len[b];
+            // this group's sequence: the unit's member hg (PAIR), else the tile's sequence
+            const int seq = PAIR ? NM * b + hg : b;
+            const bool seq_ok = seq < P.batch;
+            const int len = seq_ok ? P.len[seq] : 0;
             const bool valid = j0 + jl < len;
             const int s = i % a.ks;
             if (!bad) bad = !mbar_wait(&u_full[i & 1], (uint32_t)((i >> 1) & 1), lim, a.err, abort);
@@ -371,13 +393,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 // With the TMA swizzle, 16-byte chunk bits 4..6 are XORed with address bits
                 // 7..9 (the tiles are 1024-aligned), so the 16 keys of a warp spread over
                 // the banks instead of hitting one or two.
-                constexpr uint32_t kRow = HH * R * 2u;
+                constexpr uint32_t kRow = HS * R * 2u;
                 const uint32_t kSw = a.asw ? 7u : 0u;
-                const uint32_t akr = smem_u32(st_ak(s)) + (uint32_t)jl * kRow;
-                const uint32_t avr = smem_u32(st_av(s)) + (uint32_t)jl * kRow;
+                const int ah0 = PAIR ? 0 : hbase;      // the group's first head in the tile
+                const uint32_t akr = smem_u32(st_ak(s, PAIR ? hg : 0)) + (uint32_t)jl * kRow;
+                const uint32_t avr = smem_u32(st_av(s, PAIR ? hg : 0)) + (uint32_t)jl * kRow;
 #pragma unroll
                 for (int h = 0; h < 16; ++h) {
-                    uint32_t ka = akr + (uint32_t)(hbase + h) * 4u, va = avr + (uint32_t)(hbase + h) * 4u;
+                    uint32_t ka = akr + (uint32_t)(ah0 + h) * 4u, va = avr + (uint32_t)(ah0 + h) * 4u;
                     ka ^= ((ka >> 7) & kSw) << 4;
                     va ^= ((va >> 7) & kSw) << 4;
                     const uint32_t kw = lds_u32(ka);
@@ -438,9 +461,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 // values need only sum_j p a^V_{j,h,s}, kept per thread (its row's rank)
 #pragma unroll
                 for (int h = 0; h < 16; ++h) {
-                    const float p = ex2(sc[h] - m[h]);
+                    // (a PAIR member can have no valid key in a whole part: m stays -inf)
+                    const float p = valid ? ex2(sc[h] - m[h]) : 0.f;
                     if (sr == 0) lp[h] += p;
-                    if (valid) acc[h] = fmaf(p, av[h], acc[h]);
+                    if (valid) acc[h] = fmaf(p, av[h], acc[h]);   // a^V past the length is not data
                 }
             } else {
                 // p and W^T (row r = K index, columns = heads), bf16 pairs of adjacent rows
@@ -479,9 +503,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             const bool last = (i == n - 1) || (P.tile_prefix[b + 1] <= g + 1);
             if (last) {
                 // part done: O^T (lane = d row), l per head, written to the workspace
-                const int part = P.first_part[b] + (c - P.c_first[b]);
-                if (!in_bounds(part >= 0 && part < P.total_parts, a.err)) bad = true;
-                float* wo = a.ws_o + (size_t)(bad ? 0 : part) * HH * DH;
+                // (c_first is per unit; an odd batch's missing member writes nothing)
+                const int part = seq_ok ? P.first_part[seq] + (c - P.c_first[b]) : 0;
+                if (!in_bounds(!seq_ok || (part >= 0 && part < P.total_parts), a.err)) bad = true;
+                const bool wr = seq_ok && !bad;
+                const int oh0 = PAIR ? 0 : hbase;        // the group's first head in the sequence
+                float* wo = a.ws_o + (size_t)(wr ? part : 0) * HS * DH;
                 if constexpr (SB) {
                     // S_{h,s} = sum_j p a^V_{j,h,s}: rows of rank s are the lanes of parity
                     // s (R = 2); sum them in the warp, then over the group's 4 warps, and
@@ -497,7 +524,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                         if (lane < R) rs[(quarter * R + lane) * 16 + h] = v;
                     }
                     bar_sync(1 + hg, 128);
-                    if (!bad && r < DH) {
+                    if (wr && r < DH) {
                         float bvr[R];
 #pragma unroll
                         for (int q = 0; q < R; ++q) bvr[q] = __bfloat162float(a.cb_v[q * DH + r]);
@@ -510,7 +537,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                                                 (rs[(2 * R + q) * 16 + h] + rs[(3 * R + q) * 16 + h]);
                                 o = fmaf(S, bvr[q], o);
                             }
-                            wo[(size_t)(hbase + h) * DH + r] = o;
+                            wo[(size_t)(oh0 + h) * DH + r] = o;
                         }
                     }
                 } else {
@@ -519,9 +546,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     uint32_t o[16];
                     tmem_ld16(lane_addr + 2u * HH + hbase, o);
                     tmem_ld_wait();
-                    if (!bad && r < DH) {
+                    if (wr && r < DH) {
 #pragma unroll
-                        for (int h = 0; h < 16; ++h) wo[(size_t)(hbase + h) * DH + r] = __uint_as_float(o[h]);
+                        for (int h = 0; h < 16; ++h) wo[(size_t)(oh0 + h) * DH + r] = __uint_as_float(o[h]);
                     }
                 }
                 float* rd = red + hg * 192;
@@ -531,10 +558,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     if (lane == 0) rd[quarter * 16 + h] = v;
                 }
                 bar_sync(1 + hg, 128);
-                if (r < 16 && !bad) {
+                if (r < 16 && wr) {
                     const float l = (rd[r] + rd[16 + r]) + (rd[32 + r] + rd[48 + r]);
-                    a.ws_ml[((size_t)part * HH + hbase + r) * 2 + 0] = m[r];
-                    a.ws_ml[((size_t)part * HH + hbase + r) * 2 + 1] = l;
+                    a.ws_ml[((size_t)part * HS + oh0 + r) * 2 + 0] = m[r];
+                    a.ws_ml[((size_t)part * HS + oh0 + r) * 2 + 1] = l;
                 }
                 bar_sync(1 + hg, 128);
                 if constexpr (!SB) {
@@ -553,14 +580,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     }
 }
 
-template <int DH, int HH, int R, bool SB>
+template <int DH, int HH, int R, bool SB, bool PAIR>
 cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const DecodePlan& plan,
                      cudaStream_t st) {
     constexpr int KT = 128 / R;
-    a.a_bytes = (uint32_t)(KT * HH * R * 2);
+    constexpr int HS = PAIR ? HH / 2 : HH;       // heads per sequence
+    constexpr int NM = PAIR ? 2 : 1;             // sequences per tile
+    if (PAIR != (plan.pairs != 0)) return cudaErrorInvalidValue;
+    a.a_bytes = (uint32_t)(KT * HS * R * 2);
     const uint32_t a_pad = (a.a_bytes + 127u) & ~127u;
     constexpr int NB = DH / 64;
-    a.kstage_bytes = ((NB * kBox + 2u * a_pad) + 1023u) & ~1023u;
+    a.kstage_bytes = ((NB * kBox + 2u * NM * a_pad) + 1023u) & ~1023u;
     // (SB: no V ring, no W^T buffers)
     const size_t fixed = 1024 + (SB ? 0 : (size_t)kVS * 2 * kBox) + (SB ? 2u : 4u) * HH * 256u +
                          (HH / 16) * 192 * sizeof(float) + 32 * 8 + 16;
@@ -579,7 +609,7 @@ cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const D
     // one box of KT keys with the 128-byte swizzle: the per-key reads of unswizzled rows
     // were 16-way (h 32) and 8-way (h 16) bank conflicts.  At h 16 a row holds two keys,
     // so the capacity must be even (else bulk copies).
-    constexpr int kpr = 128 / (HH * R * 2);      // keys per 128-byte row
+    constexpr int kpr = 128 / (HS * R * 2);      // keys per 128-byte row
     CUtensorMap tmak, tmav;
     a.asw = (c.capacity % kpr == 0) ? 1 : 0;
     if (a.asw) {
@@ -594,9 +624,9 @@ cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const D
         tmav = tmk;
     }
     constexpr int threads = 128 + 32 * 4 * (HH / 16);
-    cudaError_t e = allow_smem(reinterpret_cast<const void*>(decode_tc_kernel<DH, HH, R, SB>), (int)smem);
+    cudaError_t e = allow_smem(reinterpret_cast<const void*>(decode_tc_kernel<DH, HH, R, SB, PAIR>), (int)smem);
     if (e != cudaSuccess) return e;
-    decode_tc_kernel<DH, HH, R, SB><<<plan.n_ctas, threads, smem, st>>>(tmk, tmv, tmak, tmav, a, plan);
+    decode_tc_kernel<DH, HH, R, SB, PAIR><<<plan.n_ctas, threads, smem, st>>>(tmk, tmv, tmak, tmav, a, plan);
     return cudaGetLastError();
 }
 }  // namespace
@@ -627,15 +657,16 @@ cudaError_t launch_decode_tc(const Shape& s, const void* q_a, const void* q_b, c
     a.wait_limit = wait_limit;
     a.cb_v = static_cast<const __nv_bfloat16*>(c.b_v);
     if (s.shared) {
-        if (s.Dh == 64) return s.H == 16 ? launch_t<64, 16, 2, true>(s, a, c, plan, st)
-                                         : launch_t<64, 32, 2, true>(s, a, c, plan, st);
-        return s.H == 16 ? launch_t<128, 16, 2, true>(s, a, c, plan, st)
-                         : launch_t<128, 32, 2, true>(s, a, c, plan, st);
+        // h 16: two sequences per key tile (32 score columns), sharing its table tile
+        if (s.Dh == 64) return s.H == 16 ? launch_t<64, 32, 2, true, true>(s, a, c, plan, st)
+                                         : launch_t<64, 32, 2, true, false>(s, a, c, plan, st);
+        return s.H == 16 ? launch_t<128, 32, 2, true, true>(s, a, c, plan, st)
+                         : launch_t<128, 32, 2, true, false>(s, a, c, plan, st);
     }
-    if (s.Dh == 64) return s.H == 16 ? launch_t<64, 16, 2, false>(s, a, c, plan, st)
-                                     : launch_t<64, 32, 2, false>(s, a, c, plan, st);
-    return s.H == 16 ? launch_t<128, 16, 2, false>(s, a, c, plan, st)
-                     : launch_t<128, 32, 2, false>(s, a, c, plan, st);
+    if (s.Dh == 64) return s.H == 16 ? launch_t<64, 16, 2, false, false>(s, a, c, plan, st)
+                                     : launch_t<64, 32, 2, false, false>(s, a, c, plan, st);
+    return s.H == 16 ? launch_t<128, 16, 2, false, false>(s, a, c, plan, st)
+                     : launch_t<128, 32, 2, false, false>(s, a, c, plan, st);
 }
 
 }  // namespace tpa

@@ -78,6 +78,9 @@ inline ProjLayout proj_layout(const Shape& s, const tpa_factors& f, long long T,
 //  - tensor-core decode: a persistent grid of n_ctas CTAs walks the concatenated
 //    key tiles of all sequences; CTA c takes tiles [c*N/G, (c+1)*N/G), and each
 //    (CTA, sequence) overlap is one part; c_first[b] is the first CTA on sequence b.
+//  - paired (shared-basis decode at h 16): the walk is over units of two sequences
+//    (2u, 2u+1) that share each key tile; tile_prefix and c_first are per unit, and
+//    a unit's CTAs give each member its own consecutive parts.
 struct DecodePlan {
     int32_t len[TPA_MAX_BATCH];
     int32_t first_part[TPA_MAX_BATCH];
@@ -85,7 +88,12 @@ struct DecodePlan {
     int32_t tile_prefix[TPA_MAX_BATCH + 1];
     int32_t c_first[TPA_MAX_BATCH];
     int32_t batch, n_ctas, total_tiles, total_parts, split_len, key_tile;
+    int32_t pairs;       // units of two sequences (paired plan)
+    int32_t n_units;     // units walked: batch, or ceil(batch / 2) when paired
 };
+
+// The shared-basis decode at h 16 pairs sequences (tensor-core path only).
+inline bool decode_pairs(const Shape& s) { return s.shared && s.H == 16; }
 
 // Builds the plan for the decode kernel that handles this shape (tc = tensor-core path).
 void make_decode_plan(const Shape& s, const int32_t* lengths, int batch, bool tc,
