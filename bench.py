@@ -51,7 +51,6 @@ FLUSH_BYTES = 256 << 20          # > 126 MB L2
 PROFILED_TRAFFIC = {
     ("prefill_b8_s2048_d1024", "tpa_prefill"): 26.448e6 + 0.040e6,
     ("decode_b64_ctx32k", "tpa_decode"): 4 * (604.100e6 + 6.495e6),
-    ("kvonly_decode_b16_ctx64k_128k", "tpa_decode"): 1602374 / 428112 * (548.138e6 + 6.335e6),
     ("shared_basis_decode_b64_ctx32k", "tpa_decode"): 286.800e6 + 7.677e6,
 }
 

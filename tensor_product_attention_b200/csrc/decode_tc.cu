@@ -22,8 +22,11 @@
 //
 // Warp roles: warp 0 TMA for the K ring (b^K tiles, 128-byte swizzle, and a^K/a^V),
 // warp 2 TMA for the V ring (b^V tiles), warp 1 TMEM owner and QK issuer, warp 3 PV
-// issuer, warps 4.. softmax (4 warps per 16 heads; TMEM lane = row).  TMEM: U^T
-// double-buffered (2 x h columns) and O^T (h).
+// issuer, warps 4.. softmax (4 warps per 16 heads; TMEM lane = row).  At h 32 (two
+// head groups) warp 1 issues both QK and PV and the softmax starts at warp 3: the
+// 352-thread CTA keeps a register cap of 186 (a fourth control warp measured 4% slower
+// there, while at h 16 the separate PV issuer gains 5%).  TMEM: U^T double-buffered
+// (2 x h columns) and O^T (h).
 //
 // Shared basis (B_K, B_V shared across tokens, same page, 优点与创新 5), kernel SB: b^K
 // tiles come from the layer's per-position table (row j = the key basis rotated at j,
@@ -81,7 +84,7 @@ struct TileWalk {
 };
 
 template <int DH, int HH, int R, bool SB, bool PAIR>
-__global__ void __launch_bounds__(128 + 32 * 4 * (HH / 16), 1)
+__global__ void __launch_bounds__(((HH == 32 && !SB) ? 96 : 128) + 32 * 4 * (HH / 16), 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                  const __grid_constant__ CUtensorMap tmak, const __grid_constant__ CUtensorMap tmav,
                  const DecodeTcArgs a, const DecodePlan P) {
@@ -95,6 +98,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     static_assert(!PAIR || (SB && HH == 32), "pairs: shared-basis kernel, two sequences of 16 heads");
     constexpr int HS = PAIR ? HH / 2 : HH;      // heads per sequence
     constexpr int NM = PAIR ? 2 : 1;            // sequences per tile
+    constexpr bool ONE = HH == 32 && !SB;       // h 32 contextual: one issuer warp
+    constexpr int kSoft0 = ONE ? 3 : 4;         // first softmax warp
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -151,7 +156,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         }
         mbar_init(o_done, 1);
         mbar_init(o_free, NSM);
-        mbar_init(fin, SB ? 1 : 2);              // one commit from each MMA issuer
+        mbar_init(fin, (SB || ONE) ? 1 : 2);     // one commit from each MMA issuer
         *abort = 0;
         fence_mbar_init();
     }
@@ -225,13 +230,84 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     drain_wait(&full[s], (uint32_t)((fills - 1) & 1));
             }
         }
-    } else if (warp == 1 || (warp == 3 && !SB)) {
+    } else if (warp == 1 || (warp == 3 && !SB && !ONE)) {
         // ---------------------------------------------------------------- MMA issuers
         // warp 1: QK of every tile; warp 3: PV of every tile.  A thread that polls an
         // mbarrier stalls until its own MMAs have completed, so one issuer for both
         // serialised them (QK(t+1), drain, PV(t), drain); two let the waits of one
         // overlap the MMAs of the other.
         if (lane == 0 && n > 0) {
+            if constexpr (ONE) {
+            // one issuer for both streams: QK(i), then PV(i-1); at a sequence boundary the
+            // previous part's last PV goes first (the softmax reads that part's O^T
+            // before it builds the next q~)
+            const uint32_t idesc_qk = idesc_bf16(128, HH, 0, 0);
+            const uint32_t idesc_pv = idesc_bf16(128, HH, 1, 0);
+            const uint32_t q0 = smem_u32(qbuf), w0 = smem_u32(wbuf);
+            TileWalk<KT> twq, twp;
+            twq.init(P, g0);
+            twp.init(P, g0);
+            int segq = -1, segp = -1;
+            int prev_bq = -1, prev_bp = -1;
+            auto issue_pv = [&](int j) -> bool {
+                const int g = g0 + j;
+                twp.advance(P, g);
+                const bool first = twp.b != prev_bp;
+                if (first) { ++segp; prev_bp = twp.b; }
+                const bool last = (j == n - 1) || (P.tile_prefix[twp.b + 1] <= g + 1);
+                if (!mbar_wait(&w_full[j & 1], (uint32_t)((j >> 1) & 1), lim, a.err, abort)) return false;
+                if (first && segp > 0 &&
+                    !mbar_wait(o_free, (uint32_t)((segp - 1) & 1), lim, a.err, abort))
+                    return false;
+                const int s = j % kVS;
+                if (!mbar_wait(&v_full[s], (uint32_t)((j / kVS) & 1), lim, a.err, abort)) return false;
+                tc_fence_after();
+                const uint32_t bv = smem_u32(st_bv(s));
+                const uint32_t wb = w0 + (uint32_t)(j & 1) * kQW;
+#pragma unroll
+                for (int k = 0; k < 128 / 16; ++k) {
+                    mma_ss(tmem + 2u * HH, smem_desc(bv + (uint32_t)k * 2048u, kBox, 1024, kSwizzle128),
+                           smem_desc(wb + (uint32_t)(k >> 2) * (HH * 128u) + (uint32_t)(k & 3) * 32u,
+                                     16, 1024, kSwizzle128),
+                           idesc_pv, (first && k == 0) ? 0u : 1u);
+                }
+                mma_commit(&w_empty[j & 1]);
+                mma_commit(&v_empty[s]);
+                if (last) mma_commit(o_done);
+                return true;
+            };
+            for (int i = 0; i <= n && !*abort; ++i) {
+                bool newseg = false;
+                if (i < n) {
+                    twq.advance(P, g0 + i);
+                    newseg = twq.b != prev_bq;
+                }
+                const bool pv_first = i >= 1 && (i == n || newseg);
+                if (pv_first && !issue_pv(i - 1)) break;
+                if (i < n) {
+                    if (newseg) {
+                        ++segq;
+                        prev_bq = twq.b;
+                        if (!mbar_wait(&q_ready[segq & 1], (uint32_t)((segq >> 1) & 1), lim, a.err, abort)) break;
+                    }
+                    const int s = i % a.ks;
+                    if (!mbar_wait(&k_full[s], (uint32_t)((i / a.ks) & 1), lim, a.err, abort)) break;
+                    tc_fence_after();
+                    const uint32_t bk = smem_u32(st_bk(s));
+                    const uint32_t qb = q0 + (uint32_t)(segq & 1) * kQW;
+#pragma unroll
+                    for (int k = 0; k < DH / 16; ++k) {
+                        const uint32_t cb = (uint32_t)(k >> 2), kk = (uint32_t)(k & 3) * 32u;
+                        mma_ss(tmem + (uint32_t)(i & 1) * HH,
+                               smem_desc(bk + cb * kBox + kk, 16, 1024, kSwizzle128),
+                               smem_desc(qb + cb * (HH * 128u) + kk, 16, 1024, kSwizzle128), idesc_qk,
+                               k > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&u_full[i & 1]);
+                }
+                if (i >= 1 && !pv_first && !issue_pv(i - 1)) break;
+            }
+            } else
             if (warp == 1) {
                 const uint32_t idesc_qk = idesc_bf16(128, HH, 0, 0);
                 const uint32_t q0 = smem_u32(qbuf);
@@ -300,14 +376,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             mma_commit(fin);
             drain_wait(fin, 0);
         }
-    } else if (warp >= 4) {
+    } else if (warp >= kSoft0) {
         // ---------------------------------------------------------------- softmax
-        const int sw = warp - 4;                 // 0 .. 4*NG-1
+        const int sw = warp - kSoft0;            // 0 .. 4*NG-1
         const int hg = sw >> 2;                  // head group (16 heads)
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;       // TMEM lane = tile row (key j, rank s)
         const int jl = r / R, sr = r % R;
-        const int stid = threadIdx.x - 128;      // 0 .. NSM-1
+        const int stid = threadIdx.x - 32 * kSoft0;  // 0 .. NSM-1
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
         const int hbase = hg * 16;
         float m[16], lp[16];
@@ -623,7 +699,7 @@ cudaError_t launch_t(const Shape& s, DecodeTcArgs a, const tpa_cache& c, const D
         tmak = tmk;     // unused
         tmav = tmk;
     }
-    constexpr int threads = 128 + 32 * 4 * (HH / 16);
+    constexpr int threads = ((HH == 32 && !SB) ? 96 : 128) + 32 * 4 * (HH / 16);
     cudaError_t e = allow_smem(reinterpret_cast<const void*>(decode_tc_kernel<DH, HH, R, SB, PAIR>), (int)smem);
     if (e != cudaSuccess) return e;
     decode_tc_kernel<DH, HH, R, SB, PAIR><<<plan.n_ctas, threads, smem, st>>>(tmk, tmv, tmak, tmav, a, plan);
