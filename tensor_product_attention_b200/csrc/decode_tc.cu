@@ -10,7 +10,9 @@
 //   score_h(j) = sum_s a^K_{j,h,s} U^T_{(j,s),h}      one thread per row, shfl over s
 //   W^T_{(j,s),h} = 2^(score - m_h) a^V_{j,h,s}        bf16, to shared memory
 //   O^T += b^V^T . W^T    tcgen05, M = d_h (A = b^V tile read MN-major), N = h, K = 128
-// HBM-bound: only (R_K + R_V)(h + d_h) factor elements per key are read.
+// HBM-bound: only (R_K + R_V)(h + d_h) factor elements per key are read.  Staging all
+// of them through shared memory runs at ~20 B per cycle per SM, the rate of the
+// measured HBM copy.
 //
 // Scheduling: a persistent grid of one CTA per SM walks the key tiles of all
 // sequences concatenated; CTA c takes tiles [c*N/G, (c+1)*N/G), so ragged lengths are
@@ -34,7 +36,12 @@
 // the basis b^V_s, so O_h = sum_s (sum_j p_{j,h} a^V_{j,h,s}) b^V_s: the softmax threads
 // keep sum_j p a^V in registers (each row has one rank) and apply the basis once per
 // part; there is no PV MMA, no V ring and no W^T.  Per key only the (R_K + R_V) h A
-// factors come from the sequence's cache.
+// factors come from the sequence's cache.  At h 16 (PAIR) two sequences share each
+// key tile: the stage holds one table tile and both sequences' A tiles, QK has 32
+// columns (q~ of sequence 2u in rows 0..15, of 2u+1 in rows 16..31), head group g
+// serves member g, and the plan walks units of two sequences (c_first per unit, each
+// member with its own consecutive parts).  A member with no valid key in a whole part
+// leaves m = -inf, l = 0, O = 0, which the merge weighs as zero.
 #include <algorithm>
 #include <cmath>
 
