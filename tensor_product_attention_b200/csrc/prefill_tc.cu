@@ -65,6 +65,8 @@ struct PrefillTcArgs {
     int bcap;                     // B_K / B_V rows between sequences: cap, or 0 (shared basis)
     int cache_batch;              // sequences the cache holds (bounds checks)
     long long T;                  // query rows (bounds checks)
+    int qstage;                   // the CTA's a^Q, b^Q block is bulk-copied into the last stage
+    uint32_t qa_pad;              // ... with b^Q at this offset (after a^Q, 128-aligned)
     uint32_t a_bytes;             // bytes of one a^K (or a^V) tile: KT*H*R*2
     uint32_t stage_bytes;
     float qscale, out_scale;
@@ -308,7 +310,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     uint64_t* o_done = o_ready + 2;             // [2] the last PV into O_b has completed
     uint64_t* fin = o_done + 2;                 // [2] each issuer's MMAs in flight at exit
     uint64_t* at_ready = fin + 2;               // [kATS] a transposed tile pair is written
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(at_ready + kATS);
+    uint64_t* q_full = at_ready + kATS;         // [1] the staged query block has landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 1);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -347,6 +350,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         mbar_init(&fin[0], 1);
         mbar_init(&fin[1], 1);
         for (int i = 0; i < kATS; ++i) mbar_init(&at_ready[i], 32);
+        mbar_init(q_full, 1);
         *abort = 0;
         fence_mbar_init();
     }
@@ -358,6 +362,52 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // K/V tile t into stage t % stages (the producer thread); false if an index check failed
+    auto issue_tile = [&](int t) -> bool {
+        const uint32_t full_bytes = 2u * NB * kBox;
+        const int s = t % a.stages;
+        const int j0 = t * KT;
+        const int rows_a = min(KT, a.cap - j0);
+        // the a-factor bulk copies read rows (b, j0 .. j0+rows_a) of the cache
+        if (!in_bounds(b < a.cache_batch && rows_a > 0, a.err)) { *abort = 1; return false; }
+        const uint32_t abytes = (uint32_t)rows_a * H * R * 2u;
+        mbar_arrive_expect_tx(&kv_full[s], full_bytes + 2u * abytes);
+        const int yb = b * a.bcap + j0;             // B row of key j0
+        const int y = yb * R;
+#pragma unroll
+        for (int cb = 0; cb < NB; ++cb) {
+            if constexpr (PK) {
+                // rank-major box: (column, key, rank) = (cb*64, key of j0, 0)
+                tma_load_3d(stage_bk(s) + cb * kBox, &tmk, &kv_full[s], cb * 64, yb, 0);
+                tma_load_3d(stage_bv(s) + cb * kBox, &tmv, &kv_full[s], cb * 64, yb, 0);
+            } else {
+                tma_load_2d(stage_bk(s) + cb * kBox, &tmk, &kv_full[s], cb * 64, y);
+                tma_load_2d(stage_bv(s) + cb * kBox, &tmv, &kv_full[s], cb * 64, y);
+            }
+        }
+        const long long ea = ((long long)b * a.cap + j0) * H * R;
+        bulk_load((void*)stage_ak(s), a.ca_k + ea, abytes, &kv_full[s]);
+        bulk_load((void*)stage_av(s), a.ca_v + ea, abytes, &kv_full[s]);
+        return true;
+    };
+
+    // The first K/V tiles go out before the prologue, so their latency overlaps it; with a
+    // staged query block the last stage holds the CTA's a^Q, b^Q until the prologue ends.
+    int t_pre = 0;
+    if (warp == 0 && lane == 0) {
+        if (a.qstage) {
+            const long long tq = (long long)b * a.S + q0;
+            const uint32_t qab = (uint32_t)nq * H * a.Rq * 2u, qbb = (uint32_t)nq * a.Rq * DH * 2u;
+            uint8_t* qs = stg + (size_t)(a.stages - 1) * a.stage_bytes;
+            mbar_arrive_expect_tx(q_full, qab + qbb);
+            bulk_load(qs, a.a_q + tq * H * a.Rq, qab, q_full);
+            bulk_load(qs + a.qa_pad, a.b_q + tq * a.Rq * DH, qbb, q_full);
+        }
+        const int pre = min(n_tiles, a.qstage ? a.stages - 1 : a.stages);
+        for (; t_pre < pre; ++t_pre)
+            if (!issue_tile(t_pre)) break;
+    }
+
     // ---- prologue: q~ rows by the 256 softmax threads, into TMEM (QT) or into shared
     // memory (bf16, 128-byte swizzled K-major)
     if (warp >= 4) {
@@ -367,16 +417,28 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         const long long t = (long long)b * a.S + q0 + (vq ? i_loc : 0);
         // q~ = qscale * sum_r a^Q_r b^Q_r; TPA-KVonly (Rq = 0): qscale * q[t][h][:]
         const int nr = a.Rq > 0 ? a.Rq : 1;
+        // staged: a^Q, b^Q of the CTA's queries are in shared memory (one bulk round trip
+        // instead of ~Rq * d_h / 8 dependent global loads per thread)
+        const uint8_t* qs = stg + (size_t)(a.stages - 1) * a.stage_bytes;
+        if (a.qstage) mbar_wait(q_full, 0u, lim, a.err, abort);
+        const __nv_bfloat16* aqp = a.qstage ? reinterpret_cast<const __nv_bfloat16*>(qs) + (i_loc * H + h) * a.Rq
+                                            : a.a_q + (t * H + h) * a.Rq;
+        // rank loops unrolled to the supported maximum (16) and predicated, so that aq
+        // stays in registers (a run-time trip count put it in local memory)
         float aq[16];
-        for (int r = 0; r < a.Rq; ++r) aq[r] = vq ? __bfloat162float(a.a_q[(t * H + h) * a.Rq + r]) * a.qscale : 0.f;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) aq[r] = (vq && r < a.Rq) ? __bfloat162float(aqp[r]) * a.qscale : 0.f;
         if (a.Rq == 0) aq[0] = vq ? a.qscale : 0.f;
-        const __nv_bfloat16* bq = a.Rq > 0 ? a.b_q + t * a.Rq * DH : a.b_q + (t * H + h) * DH;
+        const __nv_bfloat16* bq = a.qstage ? reinterpret_cast<const __nv_bfloat16*>(qs + a.qa_pad) + i_loc * a.Rq * DH
+                                : a.Rq > 0 ? a.b_q + t * a.Rq * DH : a.b_q + (t * H + h) * DH;
         uint32_t qw[QT ? DH / 2 : 1];
 #pragma unroll
         for (int k8 = 0; k8 < DH; k8 += 8) {
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             if (vq) {
-                for (int r = 0; r < nr; ++r) {
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    if (r >= nr) break;
                     const uint4 raw = *reinterpret_cast<const uint4*>(bq + r * DH + k8);
                     const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
@@ -413,41 +475,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
       if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            const uint32_t full_bytes = 2u * NB * kBox;
-            int t = 0;
+            int t = t_pre;                                // tiles issued before the prologue
             for (; t < n_tiles && !*abort; ++t) {
                 const int s = t % a.stages;
                 if (t >= a.stages &&
                     !mbar_wait(&kv_empty[s], (uint32_t)((t / a.stages - 1) & 1), lim, a.err, abort))
                     break;
-                const int j0 = t * KT;
-                const int rows_a = min(KT, a.cap - j0);
-                // the a-factor bulk copies read rows (b, j0 .. j0+rows_a) of the cache
-                if (!in_bounds(b < a.cache_batch && rows_a > 0, a.err)) { *abort = 1; break; }
-                const uint32_t abytes = (uint32_t)rows_a * H * R * 2u;
-                mbar_arrive_expect_tx(&kv_full[s], full_bytes + 2u * abytes);
-                const int yb = b * a.bcap + j0;             // B row of key j0
-                const int y = yb * R;
-#pragma unroll
-                for (int cb = 0; cb < NB; ++cb) {
-                    if constexpr (PK) {
-                        // rank-major box: (column, key, rank) = (cb*64, key of j0, 0)
-                        tma_load_3d(stage_bk(s) + cb * kBox, &tmk, &kv_full[s], cb * 64, yb, 0);
-                        tma_load_3d(stage_bv(s) + cb * kBox, &tmv, &kv_full[s], cb * 64, yb, 0);
-                    } else {
-                        tma_load_2d(stage_bk(s) + cb * kBox, &tmk, &kv_full[s], cb * 64, y);
-                        tma_load_2d(stage_bv(s) + cb * kBox, &tmv, &kv_full[s], cb * 64, y);
-                    }
-                }
-                const long long ea = ((long long)b * a.cap + j0) * H * R;
-                bulk_load((void*)stage_ak(s), a.ca_k + ea, abytes, &kv_full[s]);
-                bulk_load((void*)stage_av(s), a.ca_v + ea, abytes, &kv_full[s]);
+                if (!issue_tile(t)) break;
             }
             for (int s = 0; s < a.stages; ++s) {          // drain issued copies
                 const int fills = t > s ? (t - s - 1) / a.stages + 1 : 0;
                 if (fills > 0)
                     drain_wait(&kv_full[s], (uint32_t)((fills - 1) & 1));
             }
+            if (a.qstage) drain_wait(q_full, 0u);
         }
       } else if (warp <= 2) {
         // ------------------------------------------------------------ MMA issuers
@@ -774,7 +815,11 @@ cudaError_t launch_t(const PrefillTcArgs& a0, const tpa_cache& c, int batch, con
         if (!make_tmap_bf16(&tmk, c.b_k, 2, dims, stride, box) || !make_tmap_bf16(&tmv, c.b_v, 2, dims, stride, box))
             return cudaErrorInvalidValue;
     }
-    const size_t smem = 1024 + q_bytes + (size_t)a.stages * a.stage_bytes + at_bytes + (2 * a.stages + 14 + kATS) * 8 + 16;
+    // the query block (a^Q then b^Q of qpb queries) can borrow the last stage at the start
+    a.qa_pad = ((uint32_t)a.qpb * a.H * a.Rq * 2u + 127u) & ~127u;
+    a.qstage = (a.Rq > 0 && (a.H * a.Rq) % 8 == 0 &&
+                a.qa_pad + (uint32_t)a.qpb * a.Rq * DH * 2u <= a.stage_bytes) ? 1 : 0;
+    const size_t smem = 1024 + q_bytes + (size_t)a.stages * a.stage_bytes + at_bytes + (2 * a.stages + 15 + kATS) * 8 + 16;
     cudaError_t e = allow_smem(reinterpret_cast<const void*>(prefill_tc_kernel<DH, R, HC>), (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.n_qblocks, batch);
