@@ -5,6 +5,7 @@ import json
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -174,3 +175,38 @@ def test_bounds_checked_library_has_the_same_abi(bnd):
         assert "bounds-checked" in bnd.tpa_build_info()
         assert bnd.tpa_abi_version() == 2
     assert "bounds-checked" not in bnd.tpa_build_info()
+
+
+def _parts_by_overlap(unit_tiles, members, sms=148):
+    """Independent count of the tensor-core decode's parts: a persistent grid of
+    min(sms, N) CTAs splits the N concatenated unit tiles evenly (CTA c takes
+    [c*N/G, (c+1)*N/G)); every (CTA, unit) overlap gives each member sequence a part."""
+    n = sum(unit_tiles)
+    G = min(sms, n)
+    starts = np.cumsum([0] + list(unit_tiles))
+    parts = 0
+    for c in range(G):
+        lo, hi = c * n // G, (c + 1) * n // G
+        for u in range(len(unit_tiles)):
+            if starts[u] < hi and starts[u + 1] > lo:
+                parts += members[u]
+    return parts
+
+
+@pytest.mark.parametrize("lengths", [[32768] * 64, [1, 5, 30], [12000, 9001, 1, 14501], [700] * 29 + [33],
+                                     [3001], [5, 2049, 3], [65536, 1, 131072, 7, 2]])
+def test_decode_plan_parts_match_an_independent_count(bnd, lengths):
+    # The workspace holds one (m, l, o) state per (part, head); the part count of the
+    # plan built inside the library must match the overlap count above.  This runs on
+    # the host only (without a GPU the library assumes 148 SMs, as on a B200).
+    h, d, kt = 16, 128, 64
+    per_part = h * (2 + d) * 4
+    tiles = [(L + kt - 1) // kt for L in lengths]
+    ctx = bnd.Dims(0, h, d, 6, 2, 2, bnd.BF16, 0)
+    assert bnd.tpa_decode_workspace_bytes(ctx, lengths) == _parts_by_overlap(tiles, [1] * len(tiles)) * per_part
+    # shared basis at h 16: units of two sequences sharing each key tile
+    U = (len(lengths) + 1) // 2
+    unit_tiles = [max(tiles[2 * u], tiles[2 * u + 1] if 2 * u + 1 < len(tiles) else 0) for u in range(U)]
+    members = [min(2, len(lengths) - 2 * u) for u in range(U)]
+    sb = bnd.Dims(0, h, d, 6, 2, 2, bnd.BF16, 1)
+    assert bnd.tpa_decode_workspace_bytes(sb, lengths) == _parts_by_overlap(unit_tiles, members) * per_part
