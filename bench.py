@@ -254,6 +254,11 @@ class PrefillStep:
         self.ws = tpa.alloc_step_workspace(self.dims, self.pre)
         self.out_host = torch.empty(self.out.shape, dtype=tdt).pin_memory()
         self.out1_host = torch.empty(self.out1.shape, dtype=tdt).pin_memory()
+        # a second set of step inputs / outputs for the pipelined end-to-end timing
+        self.slots = [(self.x, self.xn, self.out, self.out1, self.out_host, self.out1_host),
+                      (torch.empty_like(self.x), torch.empty_like(self.xn), torch.empty_like(self.out),
+                       torch.empty_like(self.out1), torch.empty_like(self.out_host).pin_memory(),
+                       torch.empty_like(self.out1_host).pin_memory())]
         self.launches_per_step = 6   # project, append, prefill; decode step: project, decode, combine
 
     def flops(self):
@@ -263,26 +268,28 @@ class PrefillStep:
         f += attn_flops_per_pair(wl) * (causal_pairs(B, S) + B * (S + 1))
         return f
 
-    def run(self, ev: Events | None = None):
+    def run(self, ev: Events | None = None, slot: int = 0):
         t, wl, d = self.tpa, self.wl, self.dims
         B, S = wl.batch, wl.seqlen
         zero = [0] * B
+        x, xn, out, out1 = self.slots[slot][:4]
         mark = (lambda n: ev.start(n)) if ev else (lambda n: None)
         done = (lambda n: ev.stop(n)) if ev else (lambda n: None)
-        mark("project"); t.tpa_project(d, self.x, self.w, B, S, zero, self.cs, self.cap, self.fac); done("project")
+        mark("project"); t.tpa_project(d, x, self.w, B, S, zero, self.cs, self.cap, self.fac); done("project")
         mark("append"); t.tpa_cache_append(d, self.cache, self.fac, B, S, zero); done("append")
-        mark("prefill"); t.tpa_prefill(d, self.fac, self.cache, B, S, zero, self.out); done("prefill")
+        mark("prefill"); t.tpa_prefill(d, self.fac, self.cache, B, S, zero, out); done("prefill")
         mark("decode_step")
-        t.tpa_decode_step(d, self.xn, self.w, self.cs, self.cap, self.cache, self.pre, self.out1, self.ws)
+        t.tpa_decode_step(d, xn, self.w, self.cs, self.cap, self.cache, self.pre, out1, self.ws)
         done("decode_step")
 
-    def run_e2e(self):
-        """The same step from pinned host buffers: copy x in, run, copy the outputs out."""
-        self.x.copy_(self.x_host, non_blocking=True)
-        self.xn.copy_(self.xn_host, non_blocking=True)
-        self.run()
-        self.out_host.copy_(self.out, non_blocking=True)
-        self.out1_host.copy_(self.out1, non_blocking=True)
+    def e2e_inputs(self, slot):
+        """(pinned host, device) pairs each step copies in."""
+        return [(self.x_host, self.slots[slot][0]), (self.xn_host, self.slots[slot][1])]
+
+    def e2e_outputs(self, slot):
+        """(device, pinned host) pairs each step copies out."""
+        return [(self.slots[slot][2], self.slots[slot][4]), (self.slots[slot][3], self.slots[slot][5])]
+
 
     def io_bytes(self):
         h2d = self.x_host.numel() * self.x_host.element_size() + self.xn_host.numel() * self.xn_host.element_size()
@@ -328,6 +335,10 @@ class DecodeStep:
         tdt = self.dims.torch_dtype
         self.out = torch.empty((B, wl.n_heads, wl.head_dim), dtype=tdt, device="cuda")
         self.out_host = torch.empty(self.out.shape, dtype=tdt).pin_memory()
+        # a second set of step inputs / outputs for the pipelined end-to-end timing
+        like = lambda t: None if t is None else torch.empty_like(t)
+        self.slots = [(self.q_a, self.q_b, self.out, self.out_host),
+                      (like(self.q_a), like(self.q_b), like(self.out), like(self.out_host).pin_memory())]
         self.ws = tpa.alloc_workspace(self.dims, self.lengths)
         self.launches_per_step = 2   # decode, combine
 
@@ -345,19 +356,22 @@ class DecodeStep:
         q = self.q_b.numel() * self.q_b.element_size() + (0 if self.q_a is None else self.q_a.numel() * self.q_a.element_size())
         return self.factor_bytes() + q + self.out.numel() * self.out.element_size()
 
-    def run(self, ev: Events | None = None):
+    def run(self, ev: Events | None = None, slot: int = 0):
+        q_a, q_b, out = self.slots[slot][:3]
         if ev:
             ev.start("decode")
-        self.tpa.tpa_decode(self.dims, self.q_a, self.q_b, self.cache, self.lengths, self.out, self.ws)
+        self.tpa.tpa_decode(self.dims, q_a, q_b, self.cache, self.lengths, out, self.ws)
         if ev:
             ev.stop("decode")
 
-    def run_e2e(self):
-        if self.q_a is not None:
-            self.q_a.copy_(self.qa_host, non_blocking=True)
-        self.q_b.copy_(self.qb_host, non_blocking=True)
-        self.run()
-        self.out_host.copy_(self.out, non_blocking=True)
+    def e2e_inputs(self, slot):
+        pairs = [(self.qb_host, self.slots[slot][1])]
+        if self.qa_host is not None:
+            pairs.append((self.qa_host, self.slots[slot][0]))
+        return pairs
+
+    def e2e_outputs(self, slot):
+        return [(self.slots[slot][2], self.slots[slot][3])]
 
     def io_bytes(self):
         h2d = self.qb_host.numel() * self.qb_host.element_size()
@@ -414,18 +428,64 @@ def timed_legs(step, steps, flush: torch.Tensor | None):
     return ev
 
 
+class E2EPipeline:
+    """Each step copies its inputs in from pinned host memory, runs, and copies its
+    outputs out, as a serving loop would: two copy streams and two buffer sets let the
+    upload of step k+1 and the download of step k-1 overlap the compute of step k.
+    Events keep every buffer from being overwritten before it is consumed."""
+
+    def __init__(self, step):
+        self.step = step
+        self.comp = torch.cuda.current_stream()
+        self.h2d, self.d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        self.in_ready = [torch.cuda.Event(), torch.cuda.Event()]
+        self.comp_done = [torch.cuda.Event(), torch.cuda.Event()]
+        self.out_done = [torch.cuda.Event(), torch.cuda.Event()]
+        self.k = 0
+
+    def one(self):
+        s, k = self.k % 2, self.k
+        with torch.cuda.stream(self.h2d):
+            if k >= 2:
+                self.h2d.wait_event(self.comp_done[s])     # step k-2 has read these inputs
+            for host, dev in self.step.e2e_inputs(s):
+                dev.copy_(host, non_blocking=True)
+            self.in_ready[s].record(self.h2d)
+        self.comp.wait_event(self.in_ready[s])
+        if k >= 2:
+            self.comp.wait_event(self.out_done[s])         # step k-2's outputs are out
+        self.step.run(slot=s)
+        self.comp_done[s].record(self.comp)
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(self.comp_done[s])
+            for dev, host in self.step.e2e_outputs(s):
+                host.copy_(dev, non_blocking=True)
+            self.out_done[s].record(self.d2h)
+        self.k += 1
+
+    def drain(self):
+        for e in self.out_done:
+            self.comp.wait_event(e)
+
+
 def timed_e2e(step, steps, warmup, ws):
+    """End to end through the public calls, host buffers in and out every step (see
+    E2EPipeline); the events on the compute stream bracket all three streams' work."""
+    pipe = E2EPipeline(step)
     for _ in range(warmup):
-        step.run_e2e()
+        pipe.one()
     torch.cuda.synchronize()
     barrier(ws)
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record()
+    a.record(pipe.comp)
+    pipe.h2d.wait_event(a)
+    pipe.d2h.wait_event(a)
     for _ in range(steps):
-        step.run_e2e()
-    b.record()
+        pipe.one()
+    pipe.drain()
+    b.record(pipe.comp)
     torch.cuda.synchronize()
     barrier(ws)
     return max_over_ranks(ws, a.elapsed_time(b) / steps)
@@ -622,7 +682,9 @@ def main():
         "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded, workload distributions)",
         "config": config, "roofline": roof, "legs_ms": legs, "clocks": clocks,
         "e2e": {"value": e2e_v, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms},
+                "ms_per_step": e2e_ms,
+                "pipelining": "each step copies its inputs in and its outputs out (pinned host memory); "
+                              "the upload of step k+1 and the download of step k-1 overlap step k"},
         "gpu_launches": step.launches_per_step * args.steps,
     }
     del step
