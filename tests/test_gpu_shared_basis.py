@@ -182,6 +182,9 @@ DECODE_CASES = [
     (shared("sd_kv", C4), [77, 5000], 1.0, 3),
     (shared("sd_kvmulti", C4), [20000, 13001], 8.0, 3),
     (shared("sd_d64", SB, head_dim=64), [2049, 1, 700], 8.0, 3),
+    # pairs with an odd capacity (a-factor tiles by bulk copies) and the KV-only query
+    (shared("sd_kv16", SB, rank_q=0, seed=1032), [333, 4000, 17], 8.0, 3),
+    (shared("sd_odd", SB), [2049, 77, 1, 5000, 3], 1.0, 2),
 ]
 
 
