@@ -611,3 +611,77 @@ def test_shared_basis_planted_mistakes_are_caught(monkeypatch):
         return {n: np.ascontiguousarray(t[..., ::-1]) for n, t in out.items()}
     assert _pins_fail(monkeypatch, "broadcast_basis", reversed_d,
                       [test_shared_basis_forward_is_textbook_attention_on_materialised_kv]) == 1
+
+
+# -------------------------------------------------------------- brute force (scalar)
+
+def _brute_layer(x, w_cat, h, d, rq, rk, rv, base, basis=None):
+    """The TPA layer for one sequence as plain scalar loops, written from the definitions
+    (no array code): y = W x per token; factors cut in the order A_q, A_k, A_v, B_q,
+    B_k, B_v with the (head, rank) and (rank, dim) views; Q/K/V as (1/R) sums of outer
+    products (KV-only: the plain query; shared basis: B_K, B_V from ``basis``); RoPE on
+    interleaved pairs of q and k at positions 0.. ; causal softmax(q.k / sqrt(d)) v."""
+    S, D = len(x), len(x[0])
+    N = len(w_cat)
+    y = [[sum(w_cat[n][c] * x[t][c] for c in range(D)) for n in range(N)] for t in range(S)]
+    widths = [h * rq, h * rk, h * rv, (rq if rq else h) * d,
+              0 if basis else rk * d, 0 if basis else rv * d]
+    offs = [sum(widths[:i]) for i in range(6)]
+
+    def A(t, seg, hh, r, R):
+        return y[t][offs[seg] + hh * R + r]
+
+    def Bf(t, seg, r, k):
+        return y[t][offs[seg] + r * d + k]
+
+    def rot(v, p):
+        out = list(v)
+        for k in range(d // 2):
+            ang = p * base ** (-2.0 * k / d)
+            c, s = math.cos(ang), math.sin(ang)
+            out[2 * k] = v[2 * k] * c - v[2 * k + 1] * s
+            out[2 * k + 1] = v[2 * k] * s + v[2 * k + 1] * c
+        return out
+
+    Q = [[None] * h for _ in range(S)]
+    K = [[None] * h for _ in range(S)]
+    V = [[None] * h for _ in range(S)]
+    for t in range(S):
+        for hh in range(h):
+            if rq:
+                q = [sum(A(t, 0, hh, r, rq) * Bf(t, 3, r, k) for r in range(rq)) / rq for k in range(d)]
+            else:
+                q = [y[t][offs[3] + hh * d + k] for k in range(d)]
+            if basis:
+                kk = [sum(A(t, 1, hh, s, rk) * basis["b_k"][s][k] for s in range(rk)) / rk for k in range(d)]
+                vv = [sum(A(t, 2, hh, s, rv) * basis["b_v"][s][k] for s in range(rv)) / rv for k in range(d)]
+            else:
+                kk = [sum(A(t, 1, hh, s, rk) * Bf(t, 4, s, k) for s in range(rk)) / rk for k in range(d)]
+                vv = [sum(A(t, 2, hh, s, rv) * Bf(t, 5, s, k) for s in range(rv)) / rv for k in range(d)]
+            Q[t][hh], K[t][hh], V[t][hh] = rot(q, t), rot(kk, t), vv
+    out = [[[0.0] * d for _ in range(h)] for _ in range(S)]
+    for i in range(S):
+        for hh in range(h):
+            sc = [sum(Q[i][hh][k] * K[j][hh][k] for k in range(d)) / math.sqrt(d) for j in range(i + 1)]
+            mx = max(sc)
+            e = [math.exp(v - mx) for v in sc]
+            z = sum(e)
+            for k in range(d):
+                out[i][hh][k] = sum(e[j] / z * V[j][hh][k] for j in range(i + 1))
+    return out
+
+
+@pytest.mark.parametrize("rq,rk,rv,shared", [(2, 1, 2, False), (0, 2, 1, False), (3, 2, 2, True), (0, 1, 2, True)],
+                         ids=["tpa", "kvonly", "shared", "kvonly-shared"])
+def test_forward_equals_scalar_brute_force(rq, rk, rv, shared):
+    g = gen(41)
+    h, d, D, S, base = 2, 4, 6, 5, 100.0
+    dims = Dims(D, h, d, rq, rk, rv, shared_basis=shared)
+    n = sum(oracle.factor_widths(dims).values())
+    w = g.standard_normal((n, D)) / 2
+    x = g.standard_normal((1, S, D))
+    basis = {"b_k": g.standard_normal((rk, d)), "b_v": g.standard_normal((rv, d))} if shared else None
+    got, _ = oracle.tpa_forward(x, w, dims, base, basis=basis)
+    want = _brute_layer(x[0].tolist(), w.tolist(), h, d, rq, rk, rv, base,
+                        basis={k: v.tolist() for k, v in basis.items()} if shared else None)
+    assert rel(got[0], np.array(want)) < 1e-12
