@@ -210,3 +210,35 @@ def test_decode_plan_parts_match_an_independent_count(bnd, lengths):
     members = [min(2, len(lengths) - 2 * u) for u in range(U)]
     sb = bnd.Dims(0, h, d, 6, 2, 2, bnd.BF16, 1)
     assert bnd.tpa_decode_workspace_bytes(sb, lengths) == _parts_by_overlap(unit_tiles, members) * per_part
+
+
+def test_product_and_oracle_stay_apart():
+    """The product (the package, its CUDA sources and binding) never imports or reads the
+    oracle, and the oracle never imports the product; bench.py and smoke() import the
+    oracle only inside the functions that time or check it."""
+    import ast
+    pkg = os.path.join(ROOT, "tensor_product_attention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "oracle" not in text.lower() or f == "inputs.py", f
+    # inputs.py may name the oracle in prose only (it serves both sides)
+    tree = ast.parse(open(os.path.join(pkg, "inputs.py"), encoding="utf-8").read())
+    for node in ast.walk(tree):
+        if isinstance(node, (ast.Import, ast.ImportFrom)):
+            names = [a.name for a in node.names] + ([node.module] if isinstance(node, ast.ImportFrom) else [])
+            assert not any(n and n.split(".")[0] == "oracle" for n in names)
+    for f in os.listdir(os.path.join(ROOT, "oracle")):
+        if f.endswith(".py"):
+            tree = ast.parse(open(os.path.join(ROOT, "oracle", f), encoding="utf-8").read())
+            for node in ast.walk(tree):
+                if isinstance(node, (ast.Import, ast.ImportFrom)):
+                    names = [a.name for a in node.names] + ([node.module] if isinstance(node, ast.ImportFrom) else [])
+                    assert not any(n and n.split(".")[0] == "tensor_product_attention_b200" for n in names), f
+    for f in ("bench.py", "__graft_entry__.py"):
+        tree = ast.parse(open(os.path.join(ROOT, f), encoding="utf-8").read())
+        for node in tree.body:                       # module level: no oracle import
+            if isinstance(node, (ast.Import, ast.ImportFrom)):
+                names = [a.name for a in node.names] + ([node.module] if isinstance(node, ast.ImportFrom) else [])
+                assert not any(n and n.split(".")[0] == "oracle" for n in names), f
