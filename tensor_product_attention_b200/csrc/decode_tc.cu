@@ -239,10 +239,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         }
     } else if (warp == 1 || (warp == 3 && !SB && !ONE)) {
         // ---------------------------------------------------------------- MMA issuers
-        // warp 1: QK of every tile; warp 3: PV of every tile.  A thread that polls an
-        // mbarrier stalls until its own MMAs have completed, so one issuer for both
-        // serialised them (QK(t+1), drain, PV(t), drain); two let the waits of one
-        // overlap the MMAs of the other.
+        // h 16: warp 1 issues QK of every tile, warp 3 PV of every tile.  A thread that
+        // polls an mbarrier stalls until its own MMAs have completed, so one issuer for
+        // both serialised them (QK(t+1), drain, PV(t), drain); two let the waits of one
+        // overlap the MMAs of the other.  h 32 (ONE): warp 1 issues both, which keeps
+        // the CTA at three control warps.  Shared basis: warp 1 issues QK only.
         if (lane == 0 && n > 0) {
             if constexpr (ONE) {
             // one issuer for both streams: QK(i), then PV(i-1); at a sequence boundary the
