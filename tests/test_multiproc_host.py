@@ -71,3 +71,24 @@ def test_bench_accounting_matches_the_closed_forms():
     assert bench.cache_bytes_per_token(sb) == (2 + 2) * 16 * 2 == 128
     # shared basis: W_B_k and W_B_v are not projected
     assert bench.proj_flops(I.custom("p", c2, shared_basis=True), 10) == 2 * 10 * (800 - 4 * 64) * 1024
+
+
+def test_reference_arm_prints_one_contract_line():
+    """bench.py --impl reference times the fp64 oracle on the host cores and prints one
+    JSON line with the bench contract's keys (no GPU involved)."""
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=600,
+                       cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["higher_is_better"] is True and d["n_gpus"] == 1
+    assert d["value"] > 0 and d["unit"] == "TFLOP/s" and d["config"]["workload"] == "prefill_b8_s2048_d1024"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["e2e"]["value"] == d["value"]
