@@ -16,7 +16,8 @@
  *    pointers marked "host" point to host memory read before the call returns.
  *    The caller owns every buffer; the library allocates nothing and keeps no
  *    pointer after the call returns.  Its only global state is one 32-bit device
- *    error word per device (tpa_get_device_error).
+ *    error word per device (tpa_get_device_error) and the fixed scratch array of
+ *    tpa_decode_static, both file-scope device variables of the library.
  *  - Every compute call is asynchronous on `stream` (a cudaStream_t; NULL means the
  *    legacy default stream).  Arguments are validated on the host before any launch;
  *    a call that returns an error has launched nothing.  TPA_ERR_CUDA means a launch
@@ -35,6 +36,11 @@
  *    behind the page's freqs_cis / apply_rotary_emb, whose body the pages do not print).
  *  - Kernels never trap.  Where a kernel waits on a barrier it gives up after a bounded
  *    number of tries, records TPA_DEVERR_TIMEOUT in the device error word and returns.
+ *    The outputs of a call for which tpa_get_device_error then reports an error are
+ *    undefined.
+ *  - The library looks up the device address of its error word (and of the
+ *    tpa_decode_static scratch array) once per device and keeps it; it must not be
+ *    used across cudaDeviceReset or any other re-creation of a device's context.
  */
 #ifndef TPA_H
 #define TPA_H
@@ -265,15 +271,37 @@ size_t tpa_decode_step_workspace_bytes(const tpa_dims* dims, const int32_t* leng
  * The split-K scratch is a file-scope device array of TPA_DECODE_STATIC_SCRATCH_BYTES
  * that every GPU loading the library holds until the process exits.  The first call
  * on each device looks up that array's address (make it before any stream capture).
- * Calls needing more scratch than the array holds (see tpa_decode_workspace_bytes)
- * return TPA_ERR_WORKSPACE before any CUDA call.  All calls on a device share the
- * array, so calls that overlap on the GPU race: keep them ordered on one stream.
- * Nothing needs clearing between calls.  Allocates nothing.  Arguments and results
- * are those of tpa_decode. */
+ * The cached address is only valid in the context it was looked up in: do not use
+ * the library across cudaDeviceReset (or any re-creation of the device's primary
+ * context).  Arguments are checked as tpa_decode checks them, with the same status
+ * codes; then calls needing more scratch than the array holds (see
+ * tpa_decode_workspace_bytes) return TPA_ERR_WORKSPACE.  Both checks come before any
+ * CUDA call.  All calls on a device share the array, so calls that overlap on the
+ * GPU race: keep them ordered on one stream.  Nothing needs clearing between calls;
+ * but when tpa_get_device_error reports an error for a call, that call's output is
+ * undefined (it may mix in partial states an earlier call left in the array).
+ * Allocates nothing.  Arguments and results are otherwise those of tpa_decode. */
 #define TPA_DECODE_STATIC_SCRATCH_BYTES (16u << 20)
 tpa_status tpa_decode_static(const tpa_dims* dims, const void* q_a, const void* q_b,
                              const tpa_cache* cache, const int32_t* lengths, int32_t batch,
                              void* out, tpa_stream_t stream);
+
+/* Which kernel family a call with these dims runs (host query, no CUDA call):
+ *   TPA_FAMILY_TENSOR_CORE  the tcgen05 / TMA kernels (bf16 shapes they cover)
+ *   TPA_FAMILY_CUDA_CORE    the CUDA-core kernels (fp32, and bf16 shapes outside the
+ *                           tensor-core kernels' limits: see each kernel's limits)
+ *   TPA_FAMILY_NONE         the dims are invalid or the call is unsupported for them
+ * call: TPA_CALL_PROJECT (tpa_project, tpa_output_project and the projection half of
+ * tpa_decode_step), TPA_CALL_PREFILL, TPA_CALL_DECODE (tpa_decode, tpa_decode_static
+ * and the decode half of tpa_decode_step).  Lets a caller or a benchmark assert that
+ * its shape takes the tensor-core path rather than learn it from a profiler. */
+#define TPA_CALL_PROJECT 0
+#define TPA_CALL_PREFILL 1
+#define TPA_CALL_DECODE 2
+#define TPA_FAMILY_NONE (-1)
+#define TPA_FAMILY_CUDA_CORE 0
+#define TPA_FAMILY_TENSOR_CORE 1
+int32_t tpa_kernel_family(const tpa_dims* dims, int32_t call);
 
 /* Synchronise `stream`, then read and clear the device error word of the current
  * device.  *code receives the TPA_DEVERR_* value (NULL allowed).  Returns TPA_OK if

@@ -33,7 +33,7 @@ EXPORTS = ("tpa_abi_version", "tpa_build_info", "tpa_status_string", "tpa_cache_
            "tpa_rope_table", "tpa_project", "tpa_cache_append", "tpa_prefill", "tpa_decode",
            "tpa_decode_workspace_bytes", "tpa_decode_static", "tpa_decode_step",
            "tpa_decode_step_workspace_bytes", "tpa_output_project", "tpa_shared_basis_tables",
-           "tpa_get_device_error", "tpa_set_wait_limit")
+           "tpa_get_device_error", "tpa_set_wait_limit", "tpa_kernel_family")
 TPA_DECODE_STATIC_SCRATCH_BYTES = 16 << 20
 
 
@@ -87,6 +87,7 @@ _sig = {
                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "tpa_get_device_error": (ctypes.c_int, [ctypes.c_void_p, _i32p]),
     "tpa_set_wait_limit": (None, [ctypes.c_uint32]),
+    "tpa_kernel_family": (ctypes.c_int32, [_P(tpa_dims), ctypes.c_int32]),
 }
 def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     for name, (res, args) in _sig.items():
@@ -350,6 +351,15 @@ def tpa_get_device_error(stream=None) -> int:
 
 def tpa_set_wait_limit(polls: int) -> None:
     _lib.tpa_set_wait_limit(int(polls))
+
+
+CALL_PROJECT, CALL_PREFILL, CALL_DECODE = 0, 1, 2
+FAMILY = {-1: "none", 0: "cuda_core", 1: "tensor_core"}
+
+
+def tpa_kernel_family(dims: Dims, call: int) -> str:
+    """'tensor_core', 'cuda_core' or 'none': the kernel family the call takes."""
+    return FAMILY[_lib.tpa_kernel_family(ctypes.byref(dims.c()), int(call))]
 
 
 def alloc_workspace(dims: Dims, lengths, device="cuda") -> torch.Tensor:

@@ -106,6 +106,24 @@ tpa_status run_decode(const Shape& s, const void* q_a, const void* q_b, const tp
 
 }  // namespace
 
+namespace tpa {
+tpa_status validate_decode(const tpa_dims* d, const void* q_a, const void* q_b,
+                           const tpa_cache* c, const int32_t* lengths, int32_t batch,
+                           const void* out) {
+    tpa_status st = check_dims(d, false);
+    if (st != TPA_OK) return st;
+    if ((st = check_cache(c, batch)) != TPA_OK) return st;
+    if (!q_b || !lengths || !out) return TPA_ERR_INVALID;
+    if (d->rank_q > 0 && (!q_a || !aligned16(q_a))) return TPA_ERR_INVALID;
+    if (!aligned16(q_b) || !aligned16(out)) return TPA_ERR_INVALID;
+    for (int b = 0; b < batch; ++b) {
+        if (lengths[b] < 1) return TPA_ERR_INVALID;
+        if (lengths[b] > c->capacity) return TPA_ERR_CAPACITY;
+    }
+    return TPA_OK;
+}
+}  // namespace tpa
+
 extern "C" {
 
 int32_t tpa_abi_version(void) { return TPA_ABI_VERSION; }
@@ -257,17 +275,9 @@ size_t tpa_decode_workspace_bytes(const tpa_dims* d, const int32_t* lengths, int
 tpa_status tpa_decode(const tpa_dims* d, const void* q_a, const void* q_b,
                       const tpa_cache* c, const int32_t* lengths, int32_t batch, void* out,
                       void* workspace, size_t workspace_bytes, tpa_stream_t stream) {
-    tpa_status st = check_dims(d, false);
+    tpa_status st = tpa::validate_decode(d, q_a, q_b, c, lengths, batch, out);
     if (st != TPA_OK) return st;
-    if ((st = check_cache(c, batch)) != TPA_OK) return st;
-    if (!q_b || !lengths || !out || !workspace) return TPA_ERR_INVALID;
-    if (d->rank_q > 0 && (!q_a || !aligned16(q_a))) return TPA_ERR_INVALID;
-    if (!aligned16(q_b) || !aligned16(out) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-        return TPA_ERR_INVALID;
-    for (int b = 0; b < batch; ++b) {
-        if (lengths[b] < 1) return TPA_ERR_INVALID;
-        if (lengths[b] > c->capacity) return TPA_ERR_CAPACITY;
-    }
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return TPA_ERR_INVALID;
     return run_decode(shape_of(*d), q_a, q_b, *c, lengths, batch, out, workspace, workspace_bytes,
                       (cudaStream_t)stream);
 }
@@ -356,6 +366,22 @@ tpa_status tpa_decode_step(const tpa_dims* d, const void* x, const void* w_cat,
     st = run_project(s, x, w_cat, batch, 1, sp, rope_cs, L, cs);
     if (st != TPA_OK) return st;
     return run_decode(s, f.a_q, f.b_q, *c, next, batch, out, wsb + qb, workspace_bytes - qb, cs);
+}
+
+int32_t tpa_kernel_family(const tpa_dims* d, int32_t call) {
+    if (check_dims(d, false) != TPA_OK) return TPA_FAMILY_NONE;
+    const Shape s = shape_of(*d);
+    switch (call) {
+        case TPA_CALL_PROJECT:
+            return project_tc_supported(s, 1) ? TPA_FAMILY_TENSOR_CORE : TPA_FAMILY_CUDA_CORE;
+        case TPA_CALL_PREFILL:
+            if (d->head_dim > 256) return TPA_FAMILY_NONE;
+            return s.bf16 && prefill_tc_supported(s) ? TPA_FAMILY_TENSOR_CORE : TPA_FAMILY_CUDA_CORE;
+        case TPA_CALL_DECODE:
+            if (s.bf16 && decode_tc_supported(s)) return TPA_FAMILY_TENSOR_CORE;
+            return (long long)s.H * s.Dh > 8192 ? TPA_FAMILY_NONE : TPA_FAMILY_CUDA_CORE;
+    }
+    return TPA_FAMILY_NONE;
 }
 
 tpa_status tpa_get_device_error(tpa_stream_t stream, int32_t* code) {

@@ -100,6 +100,12 @@ void make_decode_plan(const Shape& s, const int32_t* lengths, int batch, bool tc
                       DecodePlan* plan);
 size_t decode_workspace_bytes(const Shape& s, const DecodePlan& plan);
 
+// Every check tpa_decode makes before it looks at the workspace: dims, cache, query,
+// output and lengths.  tpa_decode_static shares it, so both return the same status.
+tpa_status validate_decode(const tpa_dims* d, const void* q_a, const void* q_b,
+                           const tpa_cache* c, const int32_t* lengths, int32_t batch,
+                           const void* out);
+
 // ---- launchers (each returns the launch's cudaError_t) ----
 cudaError_t launch_rope_table(float* cs, int max_pos, int head_dim, double base,
                               cudaStream_t st);

@@ -96,6 +96,45 @@ def test_host_validation_rejects_bad_arguments(bnd):
     assert _call(bnd, "tpa_rope_table", by(d), 0.5, 8, fake, None) == 1
 
 
+def test_static_decode_returns_the_same_status_as_decode(bnd):
+    """tpa_decode_static checks its arguments as tpa_decode does, before any CUDA call,
+    so an unsupported shape, a null query or a length past the cache gives the same
+    code from both (and the scratch array is never looked up)."""
+    by = ctypes.byref
+    fake = 0x10000
+    c = bnd.tpa_cache(fake, fake, fake, fake, fake, 2, 8)
+    cases = [
+        (bnd.Dims(64, 5000, 16, 2, 1, 1, bnd.F32), fake, [1, 1], 2),     # h > 4096: unsupported
+        (bnd.Dims(64, 4, 16, 2, 300, 1, bnd.F32), fake, [1, 1], 2),      # rank > 256: unsupported
+        (bnd.Dims(64, 4, 16, 2, 1, 1, bnd.F32), None, [1, 1], 1),        # null query: invalid
+        (bnd.Dims(64, 4, 16, 2, 1, 1, bnd.F32), fake, [9, 1], 3),        # past the capacity
+        (bnd.Dims(64, 4, 16, 2, 1, 1, bnd.F32), fake, [0, 1], 1),        # empty context
+    ]
+    for dims, q_b, lengths, want in cases:
+        d = dims.c()
+        got_ws = _call(bnd, "tpa_decode", by(d), fake, q_b, by(c), bnd._ints(lengths), 2, fake, fake,
+                       1 << 20, None)
+        got_static = _call(bnd, "tpa_decode_static", by(d), fake, q_b, by(c), bnd._ints(lengths), 2,
+                           fake, None)
+        assert got_ws == got_static == want, (dims, got_ws, got_static)
+
+
+def test_kernel_family_names_the_path_each_shape_takes(bnd):
+    # the configured bf16 layers take the tensor-core kernels for every call
+    for h, d, rq in ((16, 64, 6), (16, 128, 6), (32, 128, 0)):
+        dims = bnd.Dims(1024, h, d, rq, 2, 2, bnd.BF16)
+        for call in (bnd.CALL_PROJECT, bnd.CALL_PREFILL, bnd.CALL_DECODE):
+            assert bnd.tpa_kernel_family(dims, call) == "tensor_core", (h, d, rq, call)
+    # fp32 layers and bf16 shapes outside the tensor-core limits use the CUDA cores
+    f32 = bnd.Dims(64, 4, 16, 2, 1, 1, bnd.F32)
+    for call in (bnd.CALL_PROJECT, bnd.CALL_PREFILL, bnd.CALL_DECODE):
+        assert bnd.tpa_kernel_family(f32, call) == "cuda_core"
+    assert bnd.tpa_kernel_family(bnd.Dims(64, 8, 32, 2, 3, 3, bnd.BF16), bnd.CALL_DECODE) == "cuda_core"
+    # invalid dims or an unknown call
+    assert bnd.tpa_kernel_family(bnd.Dims(64, 4, 15, 2, 1, 1, bnd.F32), bnd.CALL_DECODE) == "none"
+    assert bnd.tpa_kernel_family(f32, 7) == "none"
+
+
 def test_decode_step_host_validation(bnd):
     d = bnd.Dims(64, 4, 16, 2, 1, 1, bnd.F32).c()
     by = ctypes.byref

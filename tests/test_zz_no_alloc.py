@@ -4,7 +4,9 @@ Such callers (a plug-in whose host application owns every allocation, a server t
 must not call cudaMalloc while it serves) pass only inputs and outputs; the split-K
 scratch is the library's own fixed device array.  These checks call it through the
 C ABI and compare it with tpa_decode on a caller-allocated workspace, twice in a
-row, so that the scratch left by one call is shown not to disturb the next.
+row, so that the scratch left by one call is shown not to disturb the next.  Both
+calls plan the same parts and run the same kernels in the same order, so the
+results must agree bit for bit, not only within the bf16 parity tolerance.
 
 The file is named to be collected last, so that a failure here cannot hide an
 earlier test's result in a run that stops at the first failure.
@@ -51,6 +53,7 @@ def test_static_scratch_decode_matches_workspace_decode(tpa, name, lengths):
         torch.cuda.synchronize()
         assert tpa.tpa_get_device_error() == 0
         assert rel_err(out, ref) < TOL["bf16"]
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
 
 
 def test_static_scratch_decode_rejects_more_than_its_array(tpa):
