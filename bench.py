@@ -38,6 +38,7 @@ from tensor_product_attention_b200 import inputs as I  # noqa: E402
 
 METRIC = "TPA decode factor-cache GB/s (% HBM peak); prefill TFLOP/s (% bf16 peak)"
 DEFAULT = "prefill_b8_s2048_d1024"
+LAYER_LEG = "layer_prefill_b4_s8192_d2048"
 DECODE_LEG = "decode_b64_ctx32k"
 KVONLY_DECODE_LEG = "kvonly_decode_b16_ctx64k_128k"
 SHARED_DECODE_LEG = "shared_basis_decode_b64_ctx32k"
@@ -493,6 +494,17 @@ def timed_e2e(step, steps, warmup, ws):
 
 # ------------------------------------------------------------------ CPU oracle baseline
 
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -541,21 +553,98 @@ def oracle_decode_sample(wl, n_seq: int = 1, length: int | None = None):
     return time.perf_counter() - t0, total
 
 
-def cpu_baseline(wl):
+# The bounded oracle samples: the first PREFILL_SAMPLE tokens of one sequence for the
+# prefill workloads (the fp64 scores alone are h * S^2 * 8 bytes), two whole sequences
+# for decode.  The reference arm times the same samples.
+PREFILL_SAMPLE = 2048
+PREFILL_SAMPLE_1T = 512          # the single-thread run: a quarter of the tokens
+
+
+def oracle_sample(wl, one_thread=False):
+    """(rate, unit, seconds, description) of the oracle on the workload's bounded sample."""
     if wl.kind == "prefill":
-        # a bounded sample: at most 2048 tokens of one sequence (the fp64 scores alone
-        # are h * S^2 * 8 bytes)
-        S = min(wl.seqlen, 2048)
+        S = min(wl.seqlen, PREFILL_SAMPLE_1T if one_thread else PREFILL_SAMPLE)
         dt, fl = oracle_prefill_sample(wl, 1, seqlen=S)
-        return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
-                "sample": f"fp64 oracle forward of the first {S} tokens of 1 of {wl.batch} sequences "
-                          f"({wl.seqlen} tokens each): projection, RoPE, causal attention; {dt:.1f} s"}
-    dt, by = oracle_decode_sample(wl, 2)
-    return {"value": by / dt / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"fp64 oracle decode of 2 of {wl.batch} sequences; {dt:.1f} s"}
+        return fl / dt / 1e12, "TFLOP/s", dt, (
+            f"fp64 oracle forward of the first {S} tokens of 1 of {wl.batch} sequences "
+            f"({wl.seqlen} tokens each): projection, RoPE, causal attention")
+    dt, by = oracle_decode_sample(wl, 1 if one_thread else 2)
+    return by / dt / 1e9, "GB/s", dt, f"fp64 oracle decode of {1 if one_thread else 2} of {wl.batch} sequences"
+
+
+def cpu_baseline(wl):
+    """The oracle on the host cores (all BLAS threads), plus a one-thread run."""
+    v, unit, dt, what = oracle_sample(wl)
+    out = {"value": v, "unit": unit, "cores": cpu_threads(), "kind": "oracle",
+           "sample": f"{what}; {dt:.1f} s", "cpu_model": cpu_model(), "threads": cpu_threads(),
+           "host_cpus": os.cpu_count()}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            v1, _, dt1, what1 = oracle_sample(wl, one_thread=True)
+        out["one_thread"] = {"value": v1, "unit": unit, "threads": 1, "sample": f"{what1}; {dt1:.1f} s"}
+    except ImportError:
+        out["one_thread"] = None
+    return out
 
 
 # ------------------------------------------------------------------ main
+
+def workload_config(wl, args, ws):
+    """The `config` object of the JSON line: the workload by name and shape, and how it
+    was timed.  Both arms print the same object for the same workload."""
+    timing = "CUDA-graph replay of the step" if not getattr(args, "no_graph", False) else "direct calls"
+    if wl.kind == "prefill":
+        return {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seqlen, "d_model": wl.d_model,
+                "n_heads": wl.n_heads, "head_dim": wl.head_dim, "rank_q": wl.rank_q,
+                "rank_k": wl.rank_k, "rank_v": wl.rank_v,
+                "step": "project+RoPE -> append -> causal prefill, then 1 decode token per sequence",
+                "l2": "flushed between steps (256 MiB write outside the step events)",
+                "timing": timing, "parallelism": f"dp{ws} (independent sequences per rank)"}
+    return {"workload": wl.name, "batch": wl.batch, "context": list(wl.context),
+            "n_heads": wl.n_heads, "head_dim": wl.head_dim, "rank_q": wl.rank_q,
+            "rank_k": wl.rank_k, "rank_v": wl.rank_v, "shared_basis": bool(wl.shared_basis),
+            "l2": "inputs larger than L2", "timing": timing,
+            "parallelism": f"dp{ws} (independent sequences per rank)"}
+
+
+def prefill_rooflines(wl, ev, pk):
+    """Rooflines of the prefill step's two tensor-core kernels from their per-launch
+    CUDA-event times: the causal prefill (algorithmic flops per causal pair) and the
+    factor projection (2 T N D)."""
+    pre_ms = ev.mean_ms("prefill")
+    pre_fl = attn_flops_per_pair(wl) * causal_pairs(wl.batch, wl.seqlen)
+    ach = pre_fl / (pre_ms * 1e-3) / 1e12
+    pre = {"kernel": "tpa_prefill (causal attention from factors)", "bound": "tensor",
+           "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+           "frac": ach / pk["bf16_tflops"], "traffic": PROFILED_TRAFFIC.get((wl.name, "tpa_prefill")),
+           "peak_kind": f"bf16 dense, burst, {pk['source']}",
+           "algorithmic_per_launch": f"{pre_fl:.4g} flop = {attn_flops_per_pair(wl)} flop/pair x "
+                                     f"{causal_pairs(wl.batch, wl.seqlen)} causal pairs",
+           "launch_ms": pre_ms}
+    pj_ms = ev.mean_ms("project")
+    pj_fl = proj_flops(wl, wl.batch * wl.seqlen)
+    pach = pj_fl / (pj_ms * 1e-3) / 1e12
+    proj = {"kernel": "tpa_project (factor projection GEMM + RoPE epilogue)", "bound": "tensor",
+            "achieved": pach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": pach / pk["bf16_tflops"],
+            "traffic": PROFILED_TRAFFIC.get((wl.name, "tpa_project")),
+            "peak_kind": f"bf16 dense, burst, {pk['source']}",
+            "algorithmic_per_launch": f"{pj_fl:.4g} flop = 2 T N D", "launch_ms": pj_ms}
+    return pre, proj
+
+
+def assert_tensor_core_path(tpa, wl):
+    """bf16 workloads must run on the tcgen05 kernels: the bench measures those."""
+    if wl.dtype != "bf16":
+        return
+    dims = tpa.Dims(wl.d_model or 64, wl.n_heads, wl.head_dim, wl.rank_q, wl.rank_k, wl.rank_v, tpa.BF16,
+                    int(wl.shared_basis))
+    calls = [tpa.CALL_DECODE] if wl.kind == "decode" else [tpa.CALL_PROJECT, tpa.CALL_PREFILL, tpa.CALL_DECODE]
+    for call in calls:
+        fam = tpa.tpa_kernel_family(dims, call)
+        if fam != "tensor_core":
+            raise SystemExit(f"{wl.name}: call {call} would take the {fam} kernels, not the tensor-core path")
+
 
 def run_reference(args, wl, ws, rank):
     """The fp64 oracle on the host cores, timed per step on a bounded sample."""
@@ -563,24 +652,62 @@ def run_reference(args, wl, ws, rank):
         return
     vals = []
     for _ in range(args.warmup + args.steps):
-        if wl.kind == "prefill":
-            dt, fl = oracle_prefill_sample(wl, 1, seqlen=512)
-            vals.append(fl / dt / 1e12)
-        else:
-            dt, by = oracle_decode_sample(wl, 1, length=8192)
-            vals.append(by / dt / 1e9)
+        v, unit, _, what = oracle_sample(wl)
+        vals.append(v)
     v = statistics.mean(vals[args.warmup:])
-    unit = "TFLOP/s" if wl.kind == "prefill" else "GB/s"
-    sample = ("fp64 oracle forward of one 512-token sequence per step" if wl.kind == "prefill"
-              else "fp64 oracle decode of one 8192-token sequence per step")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name},
-        "cpu_baseline": {"value": v, "unit": unit, "cores": cpu_threads(), "kind": "oracle", "sample": sample},
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, workload distributions)",
+        "config": workload_config(wl, args, ws),
+        "cpu_baseline": {"value": v, "unit": unit, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"{what}, per step", "cpu_model": cpu_model()},
         "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
+
+
+def measure_prefill(step, args, ws, pk, flush, clk_ok=True):
+    """Time one prefill workload: the graph-replayed step, per-call legs, and the
+    pipelined end-to-end step.  Returns the pieces of its JSON entry."""
+    wl = step.wl
+    ms = timed(step, args.steps, args.warmup, ws, flush, graph=not args.no_graph)
+    ev = timed_legs(step, args.steps, flush)
+    e2e_ms = timed_e2e(step, args.steps, args.warmup, ws)
+    work = step.flops()
+    pre, proj = prefill_rooflines(wl, ev, pk)
+    h2d, d2h = step.io_bytes()
+    return {
+        "value": whole_job_rate(ws, work, ms) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+        "roofline": pre, "roofline_project": proj,
+        "legs_ms": {n: round(ev.mean_ms(n), 4) for n in ("project", "append", "prefill", "decode_step")},
+        "e2e": {"value": whole_job_rate(ws, work, e2e_ms) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "pipelining": "each step copies its inputs in and its outputs out (pinned host memory); "
+                              "the upload of step k+1 and the download of step k-1 overlap step k"},
+        "gpu_launches": step.launches_per_step * args.steps,
+    }
+
+
+def measure_decode(step, args, ws, pk):
+    wl = step.wl
+    ms = timed(step, args.steps, args.warmup, ws, None, graph=not args.no_graph)
+    ev = timed_legs(step, args.steps, None)
+    e2e_ms = timed_e2e(step, args.steps, args.warmup, ws)
+    ach = step.factor_bytes() / (ev.mean_ms("decode") * 1e-3) / 1e9
+    h2d, d2h = step.io_bytes()
+    return {
+        "value": whole_job_rate(ws, step.bytes(), ms) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+        "roofline": {"kernel": "tpa_decode (split-K decode + combine)", "bound": "hbm", "achieved": ach,
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
+                     "traffic": PROFILED_TRAFFIC.get((wl.name, "tpa_decode")),
+                     "peak_kind": f"HBM copy, {pk['source']}",
+                     "algorithmic_per_launch": f"{step.factor_bytes()} factor bytes",
+                     "launch_ms": ev.mean_ms("decode")},
+        "legs_ms": {"decode": round(ev.mean_ms("decode"), 4)},
+        "e2e": {"value": whole_job_rate(ws, step.bytes(), e2e_ms) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": step.launches_per_step * args.steps,
+    }
 
 
 def main():
@@ -591,7 +718,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT, choices=sorted(I.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-decode-leg", action="store_true")
+    ap.add_argument("--no-decode-leg", action="store_true", help="skip the decode and full-layer legs")
     ap.add_argument("--no-graph", action="store_true", help="time direct calls instead of graph replays")
     ap.add_argument("--capture", action="store_true",
                     help="for an ncu capture: run --warmup untimed steps and one more, print no bench line")
@@ -615,6 +742,7 @@ def main():
     ws, rank, local = dist_setup()
     from tensor_product_attention_b200 import binding as tpa
     pk = peaks()
+    assert_tensor_core_path(tpa, wl)
 
     step = PrefillStep(wl, tpa) if wl.kind == "prefill" else DecodeStep(wl, tpa)
     if args.capture:
@@ -628,89 +756,48 @@ def main():
         return
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if wl.kind == "prefill" else None
     with ClockSampler(local) as clk:
-        ms = timed(step, args.steps, args.warmup, ws, flush, graph=not args.no_graph)
-        ev = timed_legs(step, args.steps, flush)
-        e2e_ms = timed_e2e(step, args.steps, args.warmup, ws)
+        m = measure_prefill(step, args, ws, pk, flush) if wl.kind == "prefill" else measure_decode(step, args, ws, pk)
     clocks = clk.summary()
     assert tpa.tpa_get_device_error() == 0
-
-    if wl.kind == "prefill":
-        work = step.flops()
-        value = whole_job_rate(ws, work, ms) / 1e12
-        e2e_v = whole_job_rate(ws, work, e2e_ms) / 1e12
-        unit = "TFLOP/s"
-        pre_ms = ev.mean_ms("prefill")
-        pre_fl = attn_flops_per_pair(wl) * causal_pairs(wl.batch, wl.seqlen)
-        ach = pre_fl / (pre_ms * 1e-3) / 1e12
-        roof = {"kernel": "tpa_prefill (causal attention from factors)", "bound": "tensor",
-                "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach / pk["bf16_tflops"], "traffic": PROFILED_TRAFFIC.get((wl.name, "tpa_prefill")),
-                "peak_kind": f"bf16 dense, burst, {pk['source']}",
-                "algorithmic_per_launch": f"{pre_fl:.4g} flop = {attn_flops_per_pair(wl)} flop/pair x "
-                                          f"{causal_pairs(wl.batch, wl.seqlen)} causal pairs",
-                "launch_ms": pre_ms}
-        legs = {n: round(ev.mean_ms(n), 4) for n in ("project", "append", "prefill", "decode_step")}
-        config = {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seqlen, "d_model": wl.d_model,
-                  "n_heads": wl.n_heads, "head_dim": wl.head_dim, "rank_q": wl.rank_q,
-                  "rank_k": wl.rank_k, "rank_v": wl.rank_v,
-                  "step": "project+RoPE -> append -> causal prefill, then 1 decode token per sequence",
-                  "l2": "flushed between steps (256 MiB write outside the step events)",
-                  "timing": "CUDA-graph replay of the step" if not args.no_graph else "direct calls",
-                  "parallelism": f"dp{ws} (independent sequences per rank)"}
-    else:
-        work = step.bytes()
-        value = whole_job_rate(ws, work, ms) / 1e9
-        e2e_v = whole_job_rate(ws, work, e2e_ms) / 1e9
-        unit = "GB/s"
-        ach = step.factor_bytes() / (ev.mean_ms("decode") * 1e-3) / 1e9
-        roof = {"kernel": "tpa_decode (split-K decode + combine)", "bound": "hbm", "achieved": ach,
-                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
-                "traffic": PROFILED_TRAFFIC.get((wl.name, "tpa_decode")),
-                "peak_kind": f"HBM copy, {pk['source']}",
-                "algorithmic_per_launch": f"{step.factor_bytes()} factor bytes",
-                "launch_ms": ev.mean_ms("decode")}
-        legs = {"decode": round(ev.mean_ms("decode"), 4)}
-        config = {"workload": wl.name, "batch": wl.batch, "context": list(wl.context),
-                  "n_heads": wl.n_heads, "head_dim": wl.head_dim, "rank_q": wl.rank_q,
-                  "rank_k": wl.rank_k, "rank_v": wl.rank_v, "l2": "inputs larger than L2",
-                  "timing": "CUDA-graph replay of the step" if not args.no_graph else "direct calls",
-                  "parallelism": f"dp{ws} (independent sequences per rank)"}
-    h2d, d2h = step.io_bytes()
     line = {
-        "metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": m["value"], "unit": m["unit"], "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded, workload distributions)",
-        "config": config, "roofline": roof, "legs_ms": legs, "clocks": clocks,
-        "e2e": {"value": e2e_v, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms,
-                "pipelining": "each step copies its inputs in and its outputs out (pinned host memory); "
-                              "the upload of step k+1 and the download of step k-1 overlap step k"},
-        "gpu_launches": step.launches_per_step * args.steps,
+        "config": workload_config(wl, args, ws), "roofline": m["roofline"], "legs_ms": m["legs_ms"],
+        "clocks": clocks, "e2e": m["e2e"], "gpu_launches": m["gpu_launches"],
     }
+    if "roofline_project" in m:
+        line["roofline_project"] = m["roofline_project"]
     del step
     torch.cuda.empty_cache()
 
-    # the decode configurations ride along with the prefill step as separate legs
+    # The full-layer prefill (the largest single-GPU prefill workload) and the decode
+    # workloads ride along with the default step as legs, each with its own numbers.
     legs_to_run = [] if (wl.kind != "prefill" or args.no_decode_leg) else \
-        [("decode_leg", DECODE_LEG), ("kvonly_decode_leg", KVONLY_DECODE_LEG),
-         ("shared_basis_decode_leg", SHARED_DECODE_LEG)]
+        [("layer_prefill_leg", LAYER_LEG), ("decode_leg", DECODE_LEG),
+         ("kvonly_decode_leg", KVONLY_DECODE_LEG), ("shared_basis_decode_leg", SHARED_DECODE_LEG)]
     for key, name in legs_to_run:
-        dl = I.WORKLOADS[name]
-        dstep = DecodeStep(dl, tpa)
-        dms = timed(dstep, args.steps, args.warmup, ws, None, graph=not args.no_graph)
-        dev = timed_legs(dstep, args.steps, None)
-        dval = whole_job_rate(ws, dstep.bytes(), dms) / 1e9
-        dach = dstep.factor_bytes() / (dev.mean_ms("decode") * 1e-3) / 1e9
-        line[key] = {"workload": dl.name, "value": dval, "unit": "GB/s", "ms_per_step": dms,
-                     "frac_of_hbm": dach / pk["hbm_gbs"], "factor_bytes": dstep.factor_bytes(),
-                     "traffic": PROFILED_TRAFFIC.get((dl.name, "tpa_decode")),
-                     "gpu_launches": dstep.launches_per_step * args.steps}
-        line["gpu_launches"] += dstep.launches_per_step * args.steps
-        del dstep
+        if name == wl.name:
+            continue
+        lw = I.WORKLOADS[name]
+        assert_tensor_core_path(tpa, lw)
+        lstep = PrefillStep(lw, tpa) if lw.kind == "prefill" else DecodeStep(lw, tpa)
+        with ClockSampler(local) as lclk:
+            lm = measure_prefill(lstep, args, ws, pk, flush) if lw.kind == "prefill" else measure_decode(lstep, args, ws, pk)
+        entry = {"workload": lw.name, "config": workload_config(lw, args, ws), **lm, "clocks": lclk.summary()}
+        if lw.kind == "decode":
+            entry["frac_of_hbm"] = lm["roofline"]["frac"]
+            entry["factor_bytes"] = lstep.factor_bytes()
+        line[key] = entry
+        line["gpu_launches"] += lm["gpu_launches"]
+        assert tpa.tpa_get_device_error() == 0
+        del lstep
         torch.cuda.empty_cache()
 
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
+        if "layer_prefill_leg" in line:
+            line["layer_prefill_leg"]["cpu_baseline"] = cpu_baseline(I.WORKLOADS[LAYER_LEG])
     if rank == 0:
         print(json.dumps(line))
     if ws > 1:

@@ -255,6 +255,9 @@ tpa_status tpa_prefill(const tpa_dims* d, const tpa_factors* q, const tpa_cache*
     }
     Shape s = shape_of(*d);
     cudaStream_t cs = (cudaStream_t)stream;
+    if (s.bf16 && prefill_qm_supported(s))
+        return launched(launch_prefill_qm(s, *q, *c, batch, seqlen, sp, out,
+                                          device_error_ptr(), wait_limit(), cs));
     if (s.bf16 && prefill_tc_supported(s))
         return launched(launch_prefill_tc(s, *q, *c, batch, seqlen, sp, out,
                                           device_error_ptr(), wait_limit(), cs));
@@ -376,7 +379,8 @@ int32_t tpa_kernel_family(const tpa_dims* d, int32_t call) {
             return project_tc_supported(s, 1) ? TPA_FAMILY_TENSOR_CORE : TPA_FAMILY_CUDA_CORE;
         case TPA_CALL_PREFILL:
             if (d->head_dim > 256) return TPA_FAMILY_NONE;
-            return s.bf16 && prefill_tc_supported(s) ? TPA_FAMILY_TENSOR_CORE : TPA_FAMILY_CUDA_CORE;
+            return s.bf16 && (prefill_qm_supported(s) || prefill_tc_supported(s)) ? TPA_FAMILY_TENSOR_CORE
+                                                                                   : TPA_FAMILY_CUDA_CORE;
         case TPA_CALL_DECODE:
             if (s.bf16 && decode_tc_supported(s)) return TPA_FAMILY_TENSOR_CORE;
             return (long long)s.H * s.Dh > 8192 ? TPA_FAMILY_NONE : TPA_FAMILY_CUDA_CORE;

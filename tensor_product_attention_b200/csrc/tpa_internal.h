@@ -137,6 +137,12 @@ cudaError_t launch_prefill_tc(const Shape& s, const tpa_factors& q, const tpa_ca
                               int* err, uint32_t wait_limit, cudaStream_t st);
 bool prefill_tc_supported(const Shape& s);
 
+// Query-major prefill (K and V formed per tile in shared memory); preferred where supported.
+cudaError_t launch_prefill_qm(const Shape& s, const tpa_factors& q, const tpa_cache& c,
+                              int batch, int seqlen, const SeqParams& start, void* out,
+                              int* err, uint32_t wait_limit, cudaStream_t st);
+bool prefill_qm_supported(const Shape& s);
+
 cudaError_t launch_decode_simt(const Shape& s, const void* q_a, const void* q_b,
                                const tpa_cache& c, const DecodePlan& plan, float* ws, int* err,
                                cudaStream_t st);
