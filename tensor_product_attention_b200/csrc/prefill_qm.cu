@@ -128,18 +128,6 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
     return r;
 }
 
-__device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
-    __nv_bfloat162 r = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&a),
-                               *reinterpret_cast<const __nv_bfloat162*>(&b));
-    return *reinterpret_cast<uint32_t*>(&r);
-}
-__device__ __forceinline__ uint32_t hfma2_u(uint32_t a, uint32_t b, uint32_t c) {
-    __nv_bfloat162 r = __hfma2(*reinterpret_cast<const __nv_bfloat162*>(&a),
-                               *reinterpret_cast<const __nv_bfloat162*>(&b),
-                               *reinterpret_cast<const __nv_bfloat162*>(&c));
-    return *reinterpret_cast<uint32_t*>(&r);
-}
-
 template <int D, int R>
 __global__ void __launch_bounds__(kQmThreads, 1)
 prefill_qm_kernel(const __grid_constant__ CUtensorMap tbk, const __grid_constant__ CUtensorMap tbv,
@@ -161,11 +149,11 @@ prefill_qm_kernel(const __grid_constant__ CUtensorMap tbk, const __grid_constant
     uint64_t* kx_empty = bars + 9;       // [2 w][HG] QK(w, g) of the tile has completed
     uint64_t* vx_empty = bars + 13;      // [2 w][HG] PV(w, g) ...
     uint64_t* s_full = bars + 17;        // [2] scores of query tile w are in TMEM
-    uint64_t* p_full = bars + 19;        // [2] P of query tile w is in TMEM
+    // bars + 19, 20: unused
     uint64_t* o_done = bars + 21;        // [2] the last PV of query tile w has completed
     uint64_t* fin = bars + 23;           // [2] each issuer's MMAs in flight at exit
     uint64_t* a_full = bars + 25;        // [1] a^Q (KV-only: the query tiles) has landed
-    // bars + 26: unused
+    uint64_t* pp_go = bars + 26;         // [1] query tile 0's first P is done: tile 1 may start
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 27);
     volatile int* abort = reinterpret_cast<volatile int*>(bars + 28);
 
@@ -197,10 +185,11 @@ prefill_qm_kernel(const __grid_constant__ CUtensorMap tbk, const __grid_constant
         for (int s = 0; s < 2; ++s) { mbar_init(&slot_full[s], 1); mbar_init(&slot_empty[s], 8); }
         mbar_init(q_full, 8);
         mbar_init(a_full, 1);
+        mbar_init(pp_go, 1);
         for (int g = 0; g < 2; ++g) { mbar_init(&kx_full[g], 4); mbar_init(&vx_full[g], 4); }
         for (int i = 0; i < 4; ++i) { mbar_init(&kx_empty[i], 1); mbar_init(&vx_empty[i], 1); }
         for (int w = 0; w < 2; ++w) {
-            mbar_init(&s_full[w], 1); mbar_init(&p_full[w], 4);
+            mbar_init(&s_full[w], 1);
             mbar_init(&o_done[w], 1); mbar_init(&fin[w], 1);
         }
         *abort = 0;
@@ -301,13 +290,64 @@ prefill_qm_kernel(const __grid_constant__ CUtensorMap tbk, const __grid_constant
         const float sc = a.sc;
         const uint64_t sc2 = pk2(sc, sc);
         bool alive = true;
-        // One rolled step per (key tile, head): the step's code stays small, so that the
-        // issuer's code is not pushed out of the instruction cache by the softmax's.
+        // ---- this query tile's MMAs, issued by one thread of the group (the leader)
+        // once the group's P is in TMEM: PV(k), then QK(k+1) into the same S columns
+        // (in order, so QK(k+1) writes S only after PV(k) has read P).  Descriptors are
+        // formed once: stepping K by 16 adds 32 bytes, i.e. 2 in the descriptor's address
+        // field (address / 16, no carry below 256 KB); 64-column blocks are kTile apart.
+        const bool leader = (warp & 3) == 0 && lane == 0;
+        const int K = nt * HG;                         // steps (key tile, head)
+        const uint32_t s_col = tmem + 256u * (uint32_t)w;
+        const uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
+        const uint32_t idesc_pv = idesc_bf16(128, D, 0, 1);
+        const uint64_t qd0 = smem_desc(smem_u32(smem + kQOff + (uint32_t)(w * 2) * kTile), 16, 1024, kSwizzle128);
+        const uint64_t qd1 = smem_desc(smem_u32(smem + kQOff + (uint32_t)(w * 2 + (HG - 1) * NB) * kTile), 16, 1024, kSwizzle128);
+        const uint64_t kd0 = smem_desc(smem_u32(smem + kKOff), 16, 1024, kSwizzle128);
+        const uint64_t kd1 = smem_desc(smem_u32(smem + kKOff + (uint32_t)((HG - 1) * NB) * kTile), 16, 1024, kSwizzle128);
+        const uint64_t vd0 = smem_desc(smem_u32(smem + kVOff), kTile, 1024, kSwizzle128);
+        const uint64_t vd1 = smem_desc(smem_u32(smem + kVOff + (uint32_t)((HG - 1) * NB) * kTile), kTile, 1024, kSwizzle128);
+        auto issue_qk = [&](int kq) {
+            const int gq = HG == 1 ? 0 : kq % HG;
+            const uint64_t qa = gq ? qd1 : qd0, kb = gq ? kd1 : kd0;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t off = (uint64_t)((kk >> 2) * (kTile >> 4) + (kk & 3) * 2);
+                mma_ss(s_col, qa + off, kb + off, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&s_full[w]);
+            mma_commit(&kx_empty[w * HG + gq]);
+        };
+        auto issue_pv = [&](int kp, bool last) {
+            const int jp = kp / HG, gp = HG == 1 ? 0 : kp % HG;
+            const uint64_t vb = gp ? vd1 : vd0;
+            const uint32_t o_col = s_col + 128u + (uint32_t)(gp * D);
+            mma_ts(o_col, s_col, vb, idesc_pv, jp > 0 ? 1u : 0u);
+#pragma unroll
+            for (int kk = 1; kk < 8; ++kk)
+                mma_ts(o_col, s_col + (uint32_t)kk * 8u, vb + (uint64_t)(kk * 128), idesc_pv, 1u);
+            mma_commit(&vx_empty[w * HG + gp]);
+            if (last) mma_commit(&o_done[w]);
+        };
+        int vs = -1, ks = 0;       // steps whose v (k) tiles are known written: <= vs (<= ks)
+        if (leader && K > 0) {
+            // tile 1 starts one softmax behind tile 0, so that one tile's MMAs run while
+            // the other's softmax works (pp_go has one phase: the wait cannot alias)
+            bool ok = mbar_wait(q_full, 0u, lim, a.err, abort) && mbar_wait(&kx_full[0], 0u, lim, a.err, abort);
+            if (ok && w == 1) ok = mbar_wait(pp_go, 0u, lim, a.err, abort);
+            if (ok) {
+                tc_fence_after();
+                issue_qk(0);
+            }
+        }
+        __syncwarp();        // the leader's warp reconverges before the aligned barriers below
+        // One rolled step per (key tile, head): the step's code stays small.
 #pragma unroll 1
         for (int k = 0; k < nt * HG; ++k) {
             const int j = k / HG, g = k % HG;
             const bool okw = mbar_wait(&s_full[w], (uint32_t)(k & 1), lim, a.err, abort);
-            if (__any_sync(0xffffffffu, !okw)) { alive = false; break; }
+            // the group's 128 threads vote, so they all leave together if a wait gave up
+            // (the step's second barrier below is then reached by all or by none)
+            if (bar_any(2 + w, 128, !okw)) { alive = false; break; }
             tc_fence_after();
             const int j0 = j * 128;
             const bool masked = j0 + 127 > p_first;
@@ -396,8 +436,42 @@ prefill_qm_kernel(const __grid_constant__ CUtensorMap tbk, const __grid_constant
             }
             tmem_st_wait();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[w]);
+            bar_sync(2 + w, 128);                      // the group's P (and O) is in TMEM
+            if (leader) {
+                // tile 1 may start now; released before the waits below, one of which
+                // (the next key tile) needs tile 1's first QK to have completed
+                if (w == 0 && k == 0) mbar_arrive(pp_go);
+                // The expander writes k_0, .., k_{HG-1}, v_0, .., v_{HG-1} of a tile, then
+                // the next tile's, in that order, so one wait covers both tiles a step
+                // needs: v_g of tile j for PV(k), and k of step k+1, which is written
+                // before v_g unless step k+1 starts the next tile (then after it).
+                const bool more = k + 1 < K;
+                const int k1 = k + 1;
+                const bool newtile = more && k1 % HG == 0;
+                bool ok = true;
+                if (newtile ? ks < k1 : vs < k) {
+                    if (newtile) {
+                        ok = mbar_wait(&kx_full[0], (uint32_t)((k1 / HG) & 1), lim, a.err, abort);
+                        ks = k1;
+                        vs = k;
+                    } else {
+                        ok = mbar_wait(&vx_full[g], (uint32_t)(j & 1), lim, a.err, abort);
+                        vs = k;
+                        ks = max(ks, j * HG + HG - 1);
+                    }
+                }
+                if (ok) {
+                    tc_fence_after();
+                    issue_pv(k, !more);
+                    if (more) issue_qk(k + 1);
+                }
+            }
+            __syncwarp();    // reconverge: the next step's barrier vote is warp-aligned
+        }
+        if (leader) {
+            // every MMA this thread issued completes before TMEM is released
+            mma_commit(&fin[w]);
+            drain_wait(&fin[w], 0u);
         }
         if (nt > 0) {
             const bool done_ok = alive && mbar_wait(&o_done[w], 0u, lim, a.err, abort);
@@ -452,12 +526,15 @@ prefill_qm_kernel(const __grid_constant__ CUtensorMap tbk, const __grid_constant
                 const int key = j * 128 + pp * KP + kl;
                 const bool valid = key < kv_len;
                 const uint32_t row_out = (uint32_t)(pp * KP + kl);
-                uint64_t* empty = isK ? kx_empty : vx_empty;
+
 #pragma unroll
                 for (int g = 0; g < HG; ++g) {
                     // k_g (v_g) of tile j-1 is free once the QKs (PVs) of both query tiles
-                    // that read it have completed; the other head's buffer may still be busy
+                    // that read it have completed; the other head's buffer may still be busy.
+                    // These barriers have one phase per tile, and the next phase needs the
+                    // tile written here, so a parity wait cannot be overtaken.
                     if (pp == 0 && j >= 1) {
+                        uint64_t* empty = isK ? kx_empty : vx_empty;
 #pragma unroll
                         for (int w = 0; w < 2; ++w)
                             if (j - 1 < n_w(w) &&
@@ -465,26 +542,37 @@ prefill_qm_kernel(const __grid_constant__ CUtensorMap tbk, const __grid_constant
                                 ok = false;
                     }
                     if (!ok) break;
-                    uint32_t a2[R];
-#pragma unroll
-                    for (int s2 = 0; s2 < R; ++s2) a2[s2] = bcast_bf16(araw, (g0 + g) * R + s2 - xa);
+                    // k = sum_s a_s b_s for this key and head, accumulated in fp32 (packed
+                    // pairs) and rounded to bf16 once: bf16 products and sums would round at
+                    // every rank, which costs a visible part of the error budget
                     uint8_t* dst0 = smem + (isK ? kKOff : kVOff) + (uint32_t)(g * NB) * kTile;
+                    uint64_t af[R];
+#pragma unroll
+                    for (int s2 = 0; s2 < R; ++s2) {
+                        const float av = __uint_as_float(bcast_bf16(araw, (g0 + g) * R + s2 - xa) << 16);
+                        af[s2] = pk2(av, av);
+                    }
 #pragma unroll 4
                     for (int cc = 0; cc < C::CPT; ++cc) {
                         const int c = c0 + cc;
                         const int cb = c / 8, c8 = c % 8;
-                        uint4 bv[R];
+                        uint64_t acc[4];
 #pragma unroll
-                        for (int s2 = 0; s2 < R; ++s2)
-                            bv[s2] = lds_v4(src_u + sw128_offset((uint32_t)((kl * R + s2) * NB + cb), (uint32_t)c8 * 16u));
-                        uint4 o;
-                        o.x = hmul2_u(a2[0], bv[0].x); o.y = hmul2_u(a2[0], bv[0].y);
-                        o.z = hmul2_u(a2[0], bv[0].z); o.w = hmul2_u(a2[0], bv[0].w);
+                        for (int s2 = 0; s2 < R; ++s2) {
+                            const uint4 bv = lds_v4(src_u + sw128_offset((uint32_t)((kl * R + s2) * NB + cb), (uint32_t)c8 * 16u));
+                            const uint32_t wv[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
-                        for (int s2 = 1; s2 < R; ++s2) {
-                            o.x = hfma2_u(a2[s2], bv[s2].x, o.x); o.y = hfma2_u(a2[s2], bv[s2].y, o.y);
-                            o.z = hfma2_u(a2[s2], bv[s2].z, o.z); o.w = hfma2_u(a2[s2], bv[s2].w, o.w);
+                            for (int e = 0; e < 4; ++e)
+                                acc[e] = ffma2(pk2(bf16lo(wv[e]), bf16hi(wv[e])), af[s2], s2 == 0 ? pk2(0.f, 0.f) : acc[e]);
                         }
+                        uint32_t ow[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float lo, hi;
+                            upk2(acc[e], lo, hi);
+                            ow[e] = pack_bf16(lo, hi);
+                        }
+                        uint4 o = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                         if (!valid) o = make_uint4(0, 0, 0, 0);  // keys past the cached length
                         *reinterpret_cast<uint4*>(dst0 + (uint32_t)cb * kTile + sw128_offset(row_out, (uint32_t)c8 * 16u)) = o;
                     }
@@ -502,77 +590,7 @@ prefill_qm_kernel(const __grid_constant__ CUtensorMap tbk, const __grid_constant
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegCtlQm));
         if (warp < 2) {
-            // ============================================================ MMA issuer
-            // One thread issues every MMA, query tile 0's before tile 1's at each step, so
-            // that tile 0's scores land first and the two softmax groups alternate rather
-            // than compete (two issuers would interleave their MMAs one for one and keep
-            // the groups in lockstep).
-            if (warp == 0 && lane == 0) {
-                const int K0 = n_w0 * HG, K1 = n_w1 * HG;   // steps (tile, head) per query tile
-                const uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
-                const uint32_t idesc_pv = idesc_bf16(128, D, 0, 1);
-                auto issue_qk = [&](int w, int k) {
-                    const int g = k % HG;
-                    const uint32_t s_col = tmem + 256u * (uint32_t)w;
-                    const uint32_t qa = smem_u32(smem + kQOff + (uint32_t)(w * 2 + g * NB) * kTile);
-                    const uint32_t kb = smem_u32(smem + kKOff + (uint32_t)(g * NB) * kTile);
-#pragma unroll 1
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (uint32_t)(kk >> 2) * kTile + (uint32_t)(kk & 3) * 32u;
-                        mma_ss(s_col, smem_desc(qa + off, 16, 1024, kSwizzle128),
-                               smem_desc(kb + off, 16, 1024, kSwizzle128), idesc_qk, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&s_full[w]);
-                    mma_commit(&kx_empty[w * HG + g]);
-                };
-                // O_{w,g} += P . v_g   (P: the bf16 pairs over S_w; v_g MN-major)
-                auto issue_pv = [&](int w, int k, bool last) {
-                    const int j = k / HG, g = k % HG;
-                    const uint32_t s_col = tmem + 256u * (uint32_t)w;
-                    const uint32_t vb = smem_u32(smem + kVOff + (uint32_t)(g * NB) * kTile);
-                    const uint32_t o_col = s_col + 128u + (uint32_t)(g * D);
-#pragma unroll 1
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(o_col, s_col + (uint32_t)kk * 8u,
-                               smem_desc(vb + (uint32_t)kk * 2048u, kTile, 1024, kSwizzle128), idesc_pv,
-                               (j > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(&vx_empty[w * HG + g]);
-                    if (last) mma_commit(&o_done[w]);
-                };
-                bool ok = mbar_wait(q_full, 0u, lim, a.err, abort) && mbar_wait(&kx_full[0], 0u, lim, a.err, abort);
-                if (ok) {
-                    tc_fence_after();
-                    issue_qk(0, 0);
-                    if (K1 > 0) issue_qk(1, 0);
-                }
-                int k_seen = 0, v_seen = -1;                 // last step whose k_g / v_g is known written
-                for (int k = 0; ok && k < max(K0, K1); ++k) {
-                    const int j = k / HG, g = k % HG;
-#pragma unroll 1
-                    for (int w = 0; w < 2; ++w) {
-                        const int K = w ? K1 : K0;
-                        if (k >= K || !ok) continue;
-                        const bool more = k + 1 < K;
-                        ok = mbar_wait(&p_full[w], (uint32_t)(k & 1), lim, a.err, abort);
-                        if (ok && v_seen < k) {
-                            ok = mbar_wait(&vx_full[g], (uint32_t)(j & 1), lim, a.err, abort);
-                            v_seen = k;
-                        }
-                        if (ok && more && k_seen < k + 1) {
-                            ok = mbar_wait(&kx_full[(k + 1) % HG], (uint32_t)(((k + 1) / HG) & 1), lim, a.err, abort);
-                            k_seen = k + 1;
-                        }
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(w, k, !more);
-                        // S_w is overwritten only after the PV above has read P (in order)
-                        if (more) issue_qk(w, k + 1);
-                    }
-                }
-                // every MMA issued completes before TMEM is released
-                mma_commit(&fin[0]);
-                drain_wait(&fin[0], 0u);
-            }
+            // warp 0 owns the TMEM (allocated above, released below); warps 0 and 1 idle
         } else {
             // ============================================================ producers
             const int pid = warp - 2;                   // slot pid: items pid, pid + 2, ...

@@ -21,3 +21,26 @@ def tpa():
         pytest.fail("gpu test collected on a machine without a CUDA device")
     from tensor_product_attention_b200 import binding
     return binding
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """Write the parity errors the GPU tests measured (max|gpu - oracle| / max|oracle| per
+    output tensor) as JSON: to $TPA_PARITY_LOG, else to gpurun_out/parity_errors.json when
+    that folder exists.  The worst error per test shows the headroom against 1e-2 / 1e-5."""
+    import json
+    from helpers import RECORDED
+    if not RECORDED:
+        return
+    path = os.environ.get("TPA_PARITY_LOG")
+    if not path:
+        out = os.path.join(ROOT, "gpurun_out")
+        if not os.path.isdir(out):
+            return
+        path = os.path.join(out, "parity_errors.json")
+    worst = {}
+    for r in RECORDED:
+        w = worst.setdefault(r["test"], {"worst_err": 0.0, "checks": 0})
+        w["worst_err"] = max(w["worst_err"], r["err"])
+        w["checks"] += 1
+    with open(path, "w") as f:
+        json.dump({"per_test": worst, "all": RECORDED}, f, indent=1)

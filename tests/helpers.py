@@ -2,6 +2,8 @@
 the GPU.  Holds no TPA arithmetic."""
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -16,11 +18,19 @@ def f64(t) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
+# Every error rel_err measures during a test session, with the test that measured it
+# (pytest's PYTEST_CURRENT_TEST); conftest.py writes them out at the end of the session.
+RECORDED: list = []
+
+
 def rel_err(gpu, ref) -> float:
     g, r = f64(gpu), f64(ref)
     assert g.shape == r.shape, (g.shape, r.shape)
     assert np.isfinite(g).all(), "non-finite GPU output"
-    return float(np.max(np.abs(g - r)) / max(np.max(np.abs(r)), 1e-300))
+    err = float(np.max(np.abs(g - r)) / max(np.max(np.abs(r)), 1e-300))
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").rsplit(" ", 1)[0]
+    RECORDED.append({"test": test, "err": err, "elements": int(g.size)})
+    return err
 
 
 def dims_of(wl, binding):

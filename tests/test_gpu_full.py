@@ -52,12 +52,43 @@ def test_full_layer_prefill_b4_s8192_d2048(tpa):
     _full_prefill(tpa, wl, [wl.batch - 1], _rows(wl.seqlen, 40, 2))
 
 
+def test_full_layer_prefill_rows_sharp(tpa):
+    """The 8192-token layer shape at the factor level with a x 8 (a sharp softmax over up
+    to 8192 keys), on two of its sequences: sampled query rows against the oracle on the
+    same bf16 factors, so the check isolates the attention kernel."""
+    wl = I.WORKLOADS["layer_prefill_b4_s8192_d2048"]
+    B, S = 2, wl.seqlen
+    dims = dims_of(wl, tpa)
+    cache = tpa.alloc_cache(dims, B, S, fill=float("nan"))
+    q = tpa.alloc_factors(dims, B * S, kv=False)
+    seqs = []
+    for b in range(B):
+        seq = I.prefill_factors(wl, b, S, S, a_scale=8.0)
+        fill_cache(cache, b, seq)
+        q.a_q[b * S:(b + 1) * S].copy_(seq["a_q"])
+        q.b_q[b * S:(b + 1) * S].copy_(seq["b_q"])
+        seqs.append(seq)
+    out = torch.empty((B * S, wl.n_heads, wl.head_dim), dtype=torch.bfloat16, device="cuda")
+    tpa.tpa_prefill(dims, q, cache, B, S, [0] * B, out)
+    torch.cuda.synchronize()
+    assert tpa.tpa_get_device_error() == 0
+    out = out.view(B, S, wl.n_heads, wl.head_dim)
+    od = oracle_dims(wl)
+    rows = _rows(S, 40, 11)
+    for b in range(B):
+        seq = {k: f64(v) for k, v in seqs[b].items()}
+        qf = {"a_q": seq["a_q"][rows], "b_q": seq["b_q"][rows]}
+        ref = oracle.attend_from_factors(qf, seq, od, rows)
+        err = rel_err(out[b, rows], ref)
+        assert err < TOL["bf16"], (b, err)
+
+
 def test_full_kvonly_layer_prefill_b4_s8192_d4096(tpa):
     wl = I.WORKLOADS["kvonly_layer_prefill_b4_s8192_d4096"]
     _full_prefill(tpa, wl, [wl.batch - 1], _rows(wl.seqlen, 24, 3))
 
 
-def _full_decode(tpa, wl, sample):
+def _full_decode(tpa, wl, sample, a_scale=1.0):
     dims = dims_of(wl, tpa)
     lengths = [int(v) for v in I.decode_lengths(wl)]
     B = wl.batch
@@ -72,7 +103,7 @@ def _full_decode(tpa, wl, sample):
         del cs
     q_parts = {}
     for b, L in enumerate(lengths):
-        seq = I.decode_sequence(wl, b, L)
+        seq = I.decode_sequence(wl, b, L, a_scale=a_scale)
         fill_cache(cache, b, seq)
         for k in ("a_q", "b_q", "q"):
             if k in seq:
@@ -92,7 +123,7 @@ def _full_decode(tpa, wl, sample):
     if basis is not None:
         tab = oracle.shared_basis_tables({n: f64(t) for n, t in basis.items()}, od, max(lengths), wl.rope_base)
     for b in sample:
-        seq = {k: f64(v) for k, v in I.decode_sequence(wl, b, lengths[b]).items()}
+        seq = {k: f64(v) for k, v in I.decode_sequence(wl, b, lengths[b], a_scale=a_scale).items()}
         kv = seq if tab is None else {"a_k": seq["a_k"], "a_v": seq["a_v"], **tab}
         err = rel_err(out[b], oracle.decode_attention(seq, kv, od, lengths[b]))
         assert err < TOL["bf16"], (b, lengths[b], err)
@@ -107,6 +138,18 @@ def test_full_kvonly_decode_b16_ctx64k_128k(tpa):
     wl = I.WORKLOADS["kvonly_decode_b16_ctx64k_128k"]
     lengths = I.decode_lengths(wl)
     _full_decode(tpa, wl, [int(np.argmin(lengths)), int(np.argmax(lengths))])
+
+
+# The workload scales give a nearly uniform softmax; a x 8 sharpens it at full size.
+def test_full_decode_b64_ctx32k_sharp(tpa):
+    wl = I.WORKLOADS["decode_b64_ctx32k"]
+    _full_decode(tpa, wl, [5, wl.batch - 2], a_scale=8.0)
+
+
+def test_full_kvonly_decode_b16_ctx64k_128k_sharp(tpa):
+    wl = I.WORKLOADS["kvonly_decode_b16_ctx64k_128k"]
+    lengths = I.decode_lengths(wl)
+    _full_decode(tpa, wl, [int(np.argmax(lengths))], a_scale=8.0)
 
 
 def test_full_shared_basis_decode_b64_ctx32k(tpa):
