@@ -153,7 +153,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     const uint32_t lim = a.wait_limit;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < a.ks; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], NSM); }
+        // SB: two K-side producers (table tiles, a tiles) arrive on each stage
+        for (int s = 0; s < a.ks; ++s) { mbar_init(&k_full[s], SB ? 2 : 1); mbar_init(&k_empty[s], NSM); }
         for (int s = 0; s < kVS; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&u_full[i], 1);
@@ -177,10 +178,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0 || (warp == 2 && !SB)) {
+    if (warp == 0 || warp == 2) {
         // ---------------------------------------------------------------- producers
-        // warp 0: the K ring (b^K, a^K, a^V); warp 2: the V ring (b^V)
-        const bool kside = warp == 0;
+        // warp 0: the K ring (b^K, a^K, a^V); warp 2: the V ring (b^V).  SB has no V ring:
+        // there warp 0 stages the table tiles of the K ring and warp 2 its a^K, a^V tiles,
+        // since the copies one thread issues complete one after another (~0.4K cycles
+        // each from L2) and a stage holds up to six of them.
+        const bool kside = warp == 0 || SB;
+        const bool do_b = !SB || warp == 0;     // K side: the b^K (table) boxes
+        const bool do_a = !SB || warp == 2;     // K side: the a^K, a^V tiles
         const int depth = kside ? a.ks : kVS;
         uint64_t* full = kside ? k_full : v_full;
         uint64_t* empty = kside ? k_empty : v_empty;
@@ -207,11 +213,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     // twice; its second group masks every key).
                     const int rows_a = a.asw ? KT : min(KT, a.cap - j0);
                     const uint32_t abytes = (uint32_t)rows_a * HS * R * 2u;
-                    mbar_arrive_expect_tx(&full[s], NB * kBox + 2u * NM * abytes);
-                    tma_load_2d(st_bk(s), &tmk, &full[s], 0, y);
-                    if (NB == 2) tma_load_2d(st_bk(s) + kBox, &tmk, &full[s], 64, y);
+                    mbar_arrive_expect_tx(&full[s], (do_b ? NB * kBox : 0u) + (do_a ? 2u * NM * abytes : 0u));
+                    if (do_b) {
+                        tma_load_2d(st_bk(s), &tmk, &full[s], 0, y);
+                        if (NB == 2) tma_load_2d(st_bk(s) + kBox, &tmk, &full[s], 64, y);
+                    }
 #pragma unroll
-                    for (int m = 0; m < NM; ++m) {
+                    for (int m = 0; m < NM && do_a; ++m) {
                         const int sq = (NM * b + m < a.cache_batch) ? NM * b + m : NM * b;
                         if (a.asw) {
                             const int ya = (sq * a.cap + j0) / (128 / (HS * R * 2));

@@ -7,8 +7,10 @@
 // before they are stored (B_K is cached pre-rotated, same page, 关键问题及回答 问题2).
 //
 // Persistent, warp-specialised, one CTA per SM:
-//   warp 0      TMA producer: 128x64 tiles of x and BNx64 tiles of W_cat (128-byte
-//               swizzle) into a ring of shared-memory stages
+//   warps 0, 10 TMA producers: 128x64 tiles of x (warp 0) and BNx64 tiles of W_cat
+//               (warp 10), 128-byte swizzle, into a ring of shared-memory stages.  The
+//               copies one thread issues complete one after another (~0.4K cycles each
+//               from L2), so each operand has its own issuing thread.
 //   warp 1      TMEM allocator and MMA issuer: tcgen05.mma M=128, N=BN, K=16, fp32
 //               accumulators double-buffered in TMEM (2 x 256 columns)
 //   warps 2..9  epilogue: tcgen05.ld a row per thread (two warps per row quarter,
@@ -26,7 +28,7 @@ namespace tpa {
 namespace {
 using namespace sm100;
 
-constexpr int BM = 128, BK = 64, kThreads = 320;
+constexpr int BM = 128, BK = 64, kThreads = 352;
 constexpr uint32_t kStageA = BM * BK * 2;   // 16 KiB
 
 struct ProjTcArgs {
@@ -99,7 +101,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < a.stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int s = 0; s < a.stages; ++s) { mbar_init(&full[s], 2); mbar_init(&empty[s], 1); }
         for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 8); }
         mbar_init(fin, 1);
         *abort = 0;
@@ -113,8 +115,11 @@ project_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
     const uint32_t tmem = *tmem_slot;
     const uint32_t lim = a.wait_limit;
 
-    if (warp == 0) {
+    if (warp == 0 || warp == 10) {
         if (lane == 0) {
+            // warp 0 stages the x tiles, warp 10 the W_cat tiles; each arrives once per
+            // stage with its own byte count
+            const bool xs = warp == 0;
             long long it = 0;
             for (int tile = blockIdx.x; tile < a.n_tiles && !*abort; tile += gridDim.x) {
                 const int m = tile / a.n_tiles_n, n = tile - m * a.n_tiles_n;
@@ -123,9 +128,13 @@ project_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
                     if (it >= a.stages &&
                         !mbar_wait(&empty[s], (uint32_t)((it / a.stages - 1) & 1), lim, a.err, abort))
                         break;
-                    mbar_arrive_expect_tx(&full[s], kStageA + stage_b);
-                    tma_load_2d(sa + (size_t)s * kStageA, &tmx, &full[s], kb * BK, m * BM);
-                    tma_load_2d(sb + (size_t)s * stage_b, &tmw, &full[s], kb * BK, n * a.BN);
+                    if (xs) {
+                        mbar_arrive_expect_tx(&full[s], kStageA);
+                        tma_load_2d(sa + (size_t)s * kStageA, &tmx, &full[s], kb * BK, m * BM);
+                    } else {
+                        mbar_arrive_expect_tx(&full[s], stage_b);
+                        tma_load_2d(sb + (size_t)s * stage_b, &tmw, &full[s], kb * BK, n * a.BN);
+                    }
                 }
             }
             // drain: every issued copy lands before the CTA can exit
