@@ -8,7 +8,8 @@
 // device memory.
 //
 // One CTA takes 256 queries of one sequence (two query tiles of 128 rows) and a group
-// of HG = 128/d_h heads (two at d_h 64, one at d_h 128).  Per key tile of 128 keys:
+// of HG = 128/d_h heads.  The code is written for d_h 64 (HG 2) and 128 (HG 1), but only
+// d_h 64 is dispatched here (see prefill_qm_supported).  Per key tile of 128 keys:
 //   k_{j,h} = sum_s a^K_{j,h,s} b^K_{j,s},  v_{j,h} = sum_s a^V_{j,h,s} b^V_{j,s}
 //             (bf16, formed once per tile for the group's heads, into shared memory)
 // and then, per query tile w and head h of the group:
@@ -709,7 +710,11 @@ static int qm_a_width(const Shape& s) {
 
 bool prefill_qm_supported(const Shape& s) {
     if (!s.bf16) return false;
-    if (s.Dh != 64 && s.Dh != 128) return false;
+    // d_h 64 only.  At d_h 128 a CTA holds one head (the two query tiles' O fill the
+    // TMEM), so every head re-stages and re-expands the key tiles and the kernel is
+    // bound by shared-memory traffic: measured 2.82 ms against 2.31 ms for the
+    // (query, head)-row kernel on the b4 x s8192, h 16 layer, which therefore takes it.
+    if (s.Dh != 64) return false;
     if (s.Rk != s.Rv || (s.Rk != 1 && s.Rk != 2 && s.Rk != 4)) return false;
     const int hg = 128 / s.Dh;
     if (s.H < hg || s.H % hg != 0) return false;
@@ -745,14 +750,10 @@ cudaError_t launch_prefill_qm(const Shape& s, const tpa_factors& q, const tpa_ca
     a.out_scale = 1.f / (float)s.Rv;
     a.err = err;
     a.wait_limit = wait_limit;
-    if (s.Dh == 64) {
-        if (s.Rk == 2) return launch_qm<64, 2>(a, c, start, st);
-        if (s.Rk == 1) return launch_qm<64, 1>(a, c, start, st);
-        return launch_qm<64, 4>(a, c, start, st);
-    }
-    if (s.Rk == 2) return launch_qm<128, 2>(a, c, start, st);
-    if (s.Rk == 1) return launch_qm<128, 1>(a, c, start, st);
-    return launch_qm<128, 4>(a, c, start, st);
+    if (s.Dh != 64) return cudaErrorInvalidValue;
+    if (s.Rk == 2) return launch_qm<64, 2>(a, c, start, st);
+    if (s.Rk == 1) return launch_qm<64, 1>(a, c, start, st);
+    return launch_qm<64, 4>(a, c, start, st);
 }
 
 }  // namespace tpa
