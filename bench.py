@@ -51,6 +51,7 @@ FLUSH_BYTES = 256 << 20          # > 126 MB L2
 # (traffic grows in proportion); the b8 x s2048 prefill (query-major kernel) at full size.
 PROFILED_TRAFFIC = {
     ("prefill_b8_s2048_d1024", "tpa_prefill"): 26284288 + 9728,
+    ("prefill_b8_s2048_d1024", "tpa_project"): 35785216 + 922112,
     ("decode_b64_ctx32k", "tpa_decode"): 4 * (604.100e6 + 6.495e6),
     ("kvonly_decode_b16_ctx64k_128k", "tpa_decode"): 1602374 / 428112 * (548.136e6 + 7.281e6),
     # shared-basis decode: its staging changed after the last capture (no entry: null)

@@ -85,6 +85,15 @@ def test_project_bf16_ragged(tpa, wl):
     assert max(errs.values()) < TOL["bf16"], errs
 
 
+@pytest.mark.parametrize("wl", [C2, C5], ids=["d64", "d128"])
+def test_project_bf16_many_tiles(tpa, wl):
+    """4100 tokens (more tiles than SMs, so persistent CTAs take several tiles and both
+    TMEM accumulators), a ragged last tile and two sequences at different start
+    positions: every element of all six factors against the oracle."""
+    errs = _project_case(tpa, wl, 2, 2050, [0, 3])
+    assert max(errs.values()) < TOL["bf16"], errs
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_project_kvonly(tpa, dtype):
     """TPA-KVonly: W_Q (h*d_h rows) in the W_B_q slot, rotated per head into b_q."""
@@ -376,8 +385,8 @@ def test_decode_step_fused(tpa, case):
 # ------------------------------------------------------------ output projection
 
 @pytest.mark.parametrize("wl,T", [(TINY, 64), (I.custom("wo_d64", C2, d_model=512), 301),
-                                  (I.custom("wo_d128", C5, d_model=384), 77)],
-                         ids=["f32", "bf16-d64", "bf16-d128"])
+                                  (I.custom("wo_d128", C5, d_model=384), 77), (C2, 5000)],
+                         ids=["f32", "bf16-d64", "bf16-d128", "bf16-many-tiles"])
 def test_output_project(tpa, wl, T):
     dims = dims_of(wl, tpa)
     attn = I.attn_out(wl, T).cuda()
