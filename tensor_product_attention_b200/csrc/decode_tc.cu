@@ -194,14 +194,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             TileWalk<KT> tw;
             tw.init(P, g0);
             int i = 0;
+            int s = 0;                 // ring slot i % depth
+            uint32_t ph = 0;           // (i / depth) & 1
             for (; i < n && !*abort; ++i) {
                 const int g = g0 + i;
                 tw.advance(P, g);
                 const int b = tw.b;
                 const int j0 = (g - P.tile_prefix[b]) * KT;
-                const int s = i % depth;
-                if (i >= depth &&
-                    !mbar_wait(&empty[s], (uint32_t)((i / depth - 1) & 1), lim, a.err, abort))
+                if (i >= depth && !mbar_wait(&empty[s], ph ^ 1u, lim, a.err, abort))
                     break;
                 const int y = (int)(((long long)b * a.bcap + j0) * R);
                 if (kside && !in_bounds(NM * b < a.cache_batch && j0 < a.cap, a.err)) { *abort = 1; break; }
@@ -238,6 +238,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     tma_load_2d(st_bv(s), &tmv, &full[s], 0, y);
                     tma_load_2d(st_bv(s) + kBox, &tmv, &full[s], NB == 2 ? 64 : 0, y);
                 }
+                if (++s == depth) { s = 0; ph ^= 1u; }
             }
             for (int s = 0; s < depth; ++s) {                   // drain issued copies
                 const int fills = i > s ? (i - s - 1) / depth + 1 : 0;
@@ -265,6 +266,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             twp.init(P, g0);
             int segq = -1, segp = -1;
             int prev_bq = -1, prev_bp = -1;
+            int ks = 0;                // K ring slot of tile i: i % a.ks
+            uint32_t kph = 0;          // (i / a.ks) & 1
             auto issue_pv = [&](int j) -> bool {
                 const int g = g0 + j;
                 twp.advance(P, g);
@@ -306,10 +309,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                         prev_bq = twq.b;
                         if (!mbar_wait(&q_ready[segq & 1], (uint32_t)((segq >> 1) & 1), lim, a.err, abort)) break;
                     }
-                    const int s = i % a.ks;
-                    if (!mbar_wait(&k_full[s], (uint32_t)((i / a.ks) & 1), lim, a.err, abort)) break;
+                    if (!mbar_wait(&k_full[ks], kph, lim, a.err, abort)) break;
                     tc_fence_after();
-                    const uint32_t bk = smem_u32(st_bk(s));
+                    const uint32_t bk = smem_u32(st_bk(ks));
                     const uint32_t qb = q0 + (uint32_t)(segq & 1) * kQW;
 #pragma unroll
                     for (int k = 0; k < DH / 16; ++k) {
@@ -320,6 +322,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                                k > 0 ? 1u : 0u);
                     }
                     mma_commit(&u_full[i & 1]);
+                    if (++ks == a.ks) { ks = 0; kph ^= 1u; }
                 }
                 if (i >= 1 && !pv_first && !issue_pv(i - 1)) break;
             }
@@ -330,6 +333,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                 TileWalk<KT> twq;
                 twq.init(P, g0);
                 int segq = -1, prev_bq = -1;
+                int ks = 0;            // K ring slot of tile i: i % a.ks
+                uint32_t kph = 0;      // (i / a.ks) & 1
                 for (int i = 0; i < n && !*abort; ++i) {
                     twq.advance(P, g0 + i);
                     if (twq.b != prev_bq) {
@@ -340,10 +345,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     // U buffer i&1 is free once the softmax of tile i-2 has read it
                     if (i >= 2 && !mbar_wait(&w_full[i & 1], (uint32_t)(((i >> 1) - 1) & 1), lim, a.err, abort))
                         break;
-                    const int s = i % a.ks;
-                    if (!mbar_wait(&k_full[s], (uint32_t)((i / a.ks) & 1), lim, a.err, abort)) break;
+                    if (!mbar_wait(&k_full[ks], kph, lim, a.err, abort)) break;
                     tc_fence_after();
-                    const uint32_t bk = smem_u32(st_bk(s));
+                    const uint32_t bk = smem_u32(st_bk(ks));
                     const uint32_t qb = q0 + (uint32_t)(segq & 1) * kQW;
 #pragma unroll
                     for (int k = 0; k < DH / 16; ++k) {
@@ -354,6 +358,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                                k > 0 ? 1u : 0u);
                     }
                     mma_commit(&u_full[i & 1]);
+                    if (++ks == a.ks) { ks = 0; kph ^= 1u; }
                 }
             } else {
                 const uint32_t idesc_pv = idesc_bf16(128, HH, 1, 0);
@@ -407,6 +412,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         TileWalk<KT> tw;
         if (n > 0) tw.init(P, g0);
         int seg = -1, prev_b = -1;
+        int ks = 0;                              // K ring slot of tile i: i % a.ks
+        uint32_t kph = 0;                        // (i / a.ks) & 1
         // A failed (timed-out) wait only sets `bad`; the loop is left at the end of the
         // tile by all softmax threads together (barrier 4), so that no thread is left
         // waiting at a named barrier or a warp vote that the others have skipped.
@@ -471,9 +478,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             const bool seq_ok = seq < P.batch;
             const int len = seq_ok ? P.len[seq] : 0;
             const bool valid = j0 + jl < len;
-            const int s = i % a.ks;
+            const int s = ks;                    // this tile's K stage and its fill parity
+            const uint32_t sph = kph;
+            if (++ks == a.ks) { ks = 0; kph ^= 1u; }
             if (!bad) bad = !mbar_wait(&u_full[i & 1], (uint32_t)((i >> 1) & 1), lim, a.err, abort);
-            if (!bad) bad = !mbar_wait(&k_full[s], (uint32_t)((i / a.ks) & 1), lim, a.err, abort);
+            if (!bad) bad = !mbar_wait(&k_full[s], sph, lim, a.err, abort);
             tc_fence_after();
             uint32_t u[16];
             tmem_ld16(lane_addr + (uint32_t)(i & 1) * HH + hbase, u);
