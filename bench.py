@@ -52,9 +52,9 @@ FLUSH_BYTES = 256 << 20          # > 126 MB L2
 PROFILED_TRAFFIC = {
     ("prefill_b8_s2048_d1024", "tpa_prefill"): 26284288 + 9728,
     ("prefill_b8_s2048_d1024", "tpa_project"): 35785216 + 922112,
-    ("decode_b64_ctx32k", "tpa_decode"): 4 * (604.100e6 + 6.495e6),
-    ("kvonly_decode_b16_ctx64k_128k", "tpa_decode"): 1602374 / 428112 * (548.136e6 + 7.281e6),
-    # shared-basis decode: its staging changed after the last capture (no entry: null)
+    ("decode_b64_ctx32k", "tpa_decode"): 4 * (604.104192e6 + 6.208e6),
+    ("kvonly_decode_b16_ctx64k_128k", "tpa_decode"): 1602374 / 428112 * (548.204288e6 + 9.393664e6),
+    ("shared_basis_decode_b64_ctx32k", "tpa_decode"): 287.670784e6 + 7.064576e6,
 }
 
 
