@@ -129,6 +129,36 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
     return r;
 }
 
+// 2^d for a pair of exponents on the FMA pipe, beside ex2.approx on MUFU (Cody–Waite style
+// range reduction with a fitted polynomial): d = n + f with n = round(d) -- adding 1.5 * 2^23
+// leaves n in the low mantissa bits -- and f in [-1/2, 1/2]; 2^f by a cubic whose
+// coefficients were fitted by Remez exchange to equioscillating relative error on
+// [-1/2, 1/2] (7.5e-5, evaluated in fp32 Horner form, against the 2^-9 half-ulp of the
+// bf16 P); n is then added to the exponent field.  d is clamped at -126 so that the
+// exponent field stays in range (such terms give at most 2^-126).
+constexpr float kE2C0 = 0.99992806f, kE2C1 = 0.69326097f, kE2C2 = 0.24261113f, kE2C3 = 0.05517167f;
+// Key pairs of a 32-column chunk whose exp2 runs on the FMA pipe: every kFmaExpEvery-th pair
+// (0: none).  Measured at b8 x s2048 with every 4th pair: 0.2395 ms against 0.2316 ms with
+// all of them on MUFU.  MUFU is not this kernel's bound (31% busy); the split's extra FMA
+// and integer instructions cost more issue slots than the MUFU time they save.
+constexpr int kFmaExpEvery = 0;
+[[maybe_unused]] constexpr int kFmaExpMod = kFmaExpEvery > 0 ? kFmaExpEvery : 1;
+[[maybe_unused]] __device__ __forceinline__ void ex2_fma_pair(float d0, float d1, float& p0, float& p1) {
+    constexpr float kShift = 12582912.f;   // 1.5 * 2^23
+    const uint64_t dd = pk2(fmaxf(d0, -126.f), fmaxf(d1, -126.f));
+    const uint64_t t = fadd2(dd, pk2(kShift, kShift));
+    const uint64_t n = fadd2(t, pk2(-kShift, -kShift));
+    const uint64_t f = ffma2(n, pk2(-1.f, -1.f), dd);
+    uint64_t q = ffma2(f, pk2(kE2C3, kE2C3), pk2(kE2C2, kE2C2));
+    q = ffma2(q, f, pk2(kE2C1, kE2C1));
+    q = ffma2(q, f, pk2(kE2C0, kE2C0));
+    float t0, t1, q0, q1;
+    upk2(t, t0, t1);
+    upk2(q, q0, q1);
+    p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+    p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
 template <int D, int R>
 __global__ void __launch_bounds__(kQmThreads, 1)
 prefill_qm_kernel(const __grid_constant__ CUtensorMap tbk, const __grid_constant__ CUtensorMap tbv,
@@ -399,7 +429,22 @@ prefill_qm_kernel(const __grid_constant__ CUtensorMap tbk, const __grid_constant
                         d0 = cb + 2 * q <= lim_c ? d0 : -INFINITY;
                         d1 = cb + 2 * q + 1 <= lim_c ? d1 : -INFINITY;
                     }
-                    const float p0 = ex2(d0), p1 = ex2(d1);
+                    float p0 = 0.f, p1 = 0.f;
+                    bool on_mufu = true;
+                    if constexpr (kFmaExpEvery > 0) {
+                        if (q % kFmaExpMod == kFmaExpMod - 1) {
+                            on_mufu = false;
+                            ex2_fma_pair(d0, d1, p0, p1);
+                            if (masked) {
+                                p0 = cb + 2 * q <= lim_c ? p0 : 0.f;
+                                p1 = cb + 2 * q + 1 <= lim_c ? p1 : 0.f;
+                            }
+                        }
+                    }
+                    if (on_mufu) {
+                        p0 = ex2(d0);
+                        p1 = ex2(d1);
+                    }
                     if (q & 1) sum2b = fadd2(sum2b, pk2(p0, p1));
                     else sum2a = fadd2(sum2a, pk2(p0, p1));
                     pk[q] = pack_bf16(p0, p1);
