@@ -23,7 +23,10 @@
 //               pairs.  Runs while the MMA warp fills the other accumulator.
 // The single-thread loops keep their ring position as 32-bit stage/phase counters: a
 // 64-bit modulo per k-block cost the MMA issuer more than half of the tensor rate.
-// Tensor-bound: 2*T*N*D flops; x and W_cat are read once from HBM (W_cat stays in L2).
+// Counted against the tensor peak (2*T*N*D flops); x and W_cat are read once from HBM
+// (W_cat stays in L2).  At 128x160 tiles the main loop runs near the shared-memory port
+// bound instead: per k-block the SM takes 36 KB of TMA writes and serves 36 KB of MMA
+// operand reads, ~576 cycles at 128 B/clk against 320 of MMA.
 #include <algorithm>
 #include <cstring>
 
