@@ -4,6 +4,7 @@ import sys
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+RUN_OUTPUT_DIR = "gpurun_out"   # the folder a GPU run brings back
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
@@ -25,15 +26,16 @@ def tpa():
 
 def pytest_sessionfinish(session, exitstatus):
     """Write the parity errors the GPU tests measured (max|gpu - oracle| / max|oracle| per
-    output tensor) as JSON: to $TPA_PARITY_LOG, else to gpurun_out/parity_errors.json when
-    that folder exists.  The worst error per test shows the headroom against 1e-2 / 1e-5."""
+    output tensor) as JSON: to $TPA_PARITY_LOG, else to parity_errors.json in the run-output
+    folder at the repository root when that folder exists.  The worst error per test shows
+    the headroom against 1e-2 / 1e-5."""
     import json
     from helpers import RECORDED
     if not RECORDED:
         return
     path = os.environ.get("TPA_PARITY_LOG")
     if not path:
-        out = os.path.join(ROOT, "gpurun_out")
+        out = os.path.join(ROOT, RUN_OUTPUT_DIR)
         if not os.path.isdir(out):
             return
         path = os.path.join(out, "parity_errors.json")
